@@ -1,0 +1,176 @@
+"""Seeded synthetic inputs for the attention library's tests and benchmark.
+
+This module holds no attention arithmetic: it only draws random tensors (torch CPU generator,
+fp32 normal samples, then a cast), so that the CUDA path and the fp64 oracle are fed the very same
+values. Each workload is named for what it is and its sizes, after the workloads the pages measure:
+
+* ``tiny_causal``: B=1, Hq=Hkv=2, Sq=Sk=128, D=64, causal, scale 1/8, fp32 (+ the same values in bf16).
+* ``block512``: one transformer block's attention at sequence 512 (B=4, H=16, D=64), the block the
+  "Não escreva kernels, derive-os" page times on an RTX 3090 ("Aprofundamento", second paragraph).
+* ``gqa_prefill_4k``: GQA causal prefill shaped like an 8B decoder (B=1, Hq=32, Hkv=8, S=4096,
+  D=128), standing in for the Qwen3-8B decode graph of the same paragraph.
+* ``decode48``: 48 decode streams (Hq=32, Hkv=8, D=128), per-stream cache lengths uniform in
+  [1024, 4096], packed, the 48-stream decode step of the third paragraph.
+* ``long_prefill_44k``: one 44032-token causal prefill (Hq=32, Hkv=8, D=128) with 1 % of keys given
+  a +4.0 shift on one random dimension per key, the 44k-token time-to-first-token case of the third
+  paragraph. No dataset or trained weight is used anywhere.
+
+Draw order inside one workload is fixed: Q, K, V, dO, then any structural draws (shift positions);
+the decode workload draws its lengths first, because the packed K/V size depends on them. Each
+workload uses its own generator seeded with 0 unless a seed is given.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Optional
+
+import torch
+
+
+@dataclass
+class Prefill:
+    name: str
+    q: torch.Tensor          # [B, Sq, Hq, D]
+    k: torch.Tensor          # [B, Sk, Hkv, D]
+    v: torch.Tensor          # [B, Sk, Hkv, D]
+    do: Optional[torch.Tensor]  # [B, Sq, Hq, D] or None (forward-only workload)
+    causal: bool
+    scale: float
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def dims(self):
+        B, Sq, Hq, D = self.q.shape
+        return dict(B=B, Hq=Hq, Hkv=self.k.shape[2], Sq=Sq, Sk=self.k.shape[1], D=D)
+
+
+@dataclass
+class Decode:
+    name: str
+    q: torch.Tensor          # [N, Hq, D]
+    k: torch.Tensor          # [T, Hkv, D] packed
+    v: torch.Tensor          # [T, Hkv, D] packed
+    offsets: torch.Tensor    # [N + 1] int32, offsets[0] = 0
+    scale: float
+    meta: dict = field(default_factory=dict)
+
+
+def _gen(seed: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return g
+
+
+def _randn(g: torch.Generator, *shape) -> torch.Tensor:
+    return torch.randn(*shape, generator=g, dtype=torch.float32)
+
+
+def random_prefill(B, Sq, Sk, Hq, Hkv, D, causal, dtype=torch.bfloat16, seed=0, scale=None,
+                   with_do=True, name=None) -> Prefill:
+    """i.i.d. N(0,1) Q, K, V (and dO) of the given shape, cast to ``dtype``."""
+    g = _gen(seed)
+    q = _randn(g, B, Sq, Hq, D)
+    k = _randn(g, B, Sk, Hkv, D)
+    v = _randn(g, B, Sk, Hkv, D)
+    do = _randn(g, B, Sq, Hq, D) if with_do else None
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    return Prefill(name or f"random_b{B}_sq{Sq}_sk{Sk}_hq{Hq}_hkv{Hkv}_d{D}",
+                   q.to(dtype), k.to(dtype), v.to(dtype),
+                   None if do is None else do.to(dtype), causal, scale)
+
+
+def tiny_causal(dtype=torch.float32) -> Prefill:
+    """B=1, Hq=Hkv=2, Sq=Sk=128, D=64, causal, scale 1/sqrt(64); fp32 draws from seed 0."""
+    w = random_prefill(1, 128, 128, 2, 2, 64, True, dtype=dtype, seed=0, scale=1.0 / 8.0)
+    w.name = "tiny_causal_b1_h2_s128_d64"
+    return w
+
+
+def block512(causal: bool) -> Prefill:
+    """Transformer-block attention: B=4, Hq=Hkv=16, S=512, D=64, bf16, forward and backward."""
+    w = random_prefill(4, 512, 512, 16, 16, 64, causal, seed=0)
+    w.name = f"block_b4_h16_s512_d64_{'causal' if causal else 'full'}"
+    return w
+
+
+def gqa_prefill_4k(reading: str = "A") -> Prefill:
+    """GQA causal prefill: B=1, Hq=32, Hkv=8, S=4096, D=128, bf16, forward and backward.
+
+    Q and K are i.i.d. N(0,1) "scaled by 1/sqrt(128)". Reading A (default): the tensors themselves
+    are multiplied by 128^-1/2 after sampling and the softmax scale is still 1/sqrt(D). Reading B:
+    the tensors stay N(0,1) and only the softmax scale is 1/sqrt(128).
+    """
+    g = _gen(0)
+    B, S, Hq, Hkv, D = 1, 4096, 32, 8, 128
+    q = _randn(g, B, S, Hq, D)
+    k = _randn(g, B, S, Hkv, D)
+    v = _randn(g, B, S, Hkv, D)
+    do = _randn(g, B, S, Hq, D)
+    if reading == "A":
+        q = q * (1.0 / math.sqrt(128.0))
+        k = k * (1.0 / math.sqrt(128.0))
+    elif reading != "B":
+        raise ValueError("reading must be 'A' or 'B'")
+    bf = torch.bfloat16
+    return Prefill(f"gqa_prefill_b1_hq32_hkv8_s4096_d128_causal_{reading}", q.to(bf), k.to(bf),
+                   v.to(bf), do.to(bf), True, 1.0 / math.sqrt(D), meta=dict(reading=reading))
+
+
+def long_prefill_44k(S: int = 44032, shift_fraction: float = 0.01, shift: float = 4.0) -> Prefill:
+    """Long causal prefill, forward only: B=1, Sq=Sk=S (44032), Hq=32, Hkv=8, D=128, bf16.
+
+    For each key/value head independently, round(0.01 * S) key positions are drawn without
+    replacement and each gets +4.0 on one dimension drawn uniformly in [0, 128), before the bf16
+    cast (4.0 is exact in bf16). The shifted positions are returned in ``meta['peaks']`` as
+    a list, one int64 tensor of positions per key/value head.
+    """
+    g = _gen(0)
+    B, Hq, Hkv, D = 1, 32, 8, 128
+    q = _randn(g, B, S, Hq, D)
+    k = _randn(g, B, S, Hkv, D)
+    v = _randn(g, B, S, Hkv, D)
+    n_peak = int(round(shift_fraction * S))
+    peaks = []
+    for h in range(Hkv):
+        pos = torch.randperm(S, generator=g)[:n_peak]
+        dim = torch.randint(0, D, (n_peak,), generator=g)
+        k[0, pos, h, dim] += shift
+        peaks.append(torch.sort(pos).values)
+    bf = torch.bfloat16
+    return Prefill(f"long_prefill_b1_s{S}_hq32_hkv8_d128_causal", q.to(bf), k.to(bf), v.to(bf),
+                   None, True, 1.0 / math.sqrt(D), meta=dict(peaks=peaks))
+
+
+def random_decode(N, Hq, Hkv, D, lengths, seed=0, dtype=torch.bfloat16, name=None) -> Decode:
+    """Decode batch with the given per-stream cache lengths; K/V packed [T, Hkv, D]."""
+    g = _gen(seed)
+    lengths = torch.as_tensor(lengths, dtype=torch.int64)
+    offsets = torch.zeros(N + 1, dtype=torch.int64)
+    offsets[1:] = torch.cumsum(lengths, 0)
+    T = int(offsets[-1])
+    q = _randn(g, N, Hq, D)
+    k = _randn(g, T, Hkv, D)
+    v = _randn(g, T, Hkv, D)
+    return Decode(name or f"decode_n{N}_hq{Hq}_hkv{Hkv}_d{D}", q.to(dtype), k.to(dtype),
+                  v.to(dtype), offsets.to(torch.int32), 1.0 / math.sqrt(D),
+                  meta=dict(lengths=lengths))
+
+
+def decode48(N: int = 48, lo: int = 1024, hi: int = 4096) -> Decode:
+    """48 decode streams, Hq=32, Hkv=8, D=128, bf16; lengths uniform in [1024, 4096] (seed 0).
+
+    The lengths are drawn first from the workload's generator, then Q, K, V.
+    """
+    g = _gen(0)
+    lengths = torch.randint(lo, hi + 1, (N,), generator=g)
+    offsets = torch.zeros(N + 1, dtype=torch.int64)
+    offsets[1:] = torch.cumsum(lengths, 0)
+    T = int(offsets[-1])
+    Hq, Hkv, D = 32, 8, 128
+    q = _randn(g, N, Hq, D)
+    k = _randn(g, T, Hkv, D)
+    v = _randn(g, T, Hkv, D)
+    bf = torch.bfloat16
+    return Decode(f"decode_n{N}_hq32_hkv8_d128_len{lo}-{hi}", q.to(bf), k.to(bf), v.to(bf),
+                  offsets.to(torch.int32), 1.0 / math.sqrt(D), meta=dict(lengths=lengths))

@@ -1,0 +1,269 @@
+"""fp64 NumPy oracle: scaled-dot-product attention written as its plain definition.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring for who may import it).
+
+Sources. The pages state the method only in words:
+  * "Não escreva kernels, derive-os" (ceviu.com.br), section "Aprofundamento", first paragraph:
+    flash attention is what falls out once the online softmax is recognised as a monoid, and a
+    comprehension is a reduction under a monoid whose body is a graph of scalar expressions.
+  * Same page, section "Perguntas frequentes", "O que o Tang propõe de diferente?": the backward
+    pass also comes out of rewrites of the same graph.
+  * "Tang Project Derives GPU Kernels via IR ..." (aibriefing.imbch.dev), section "Details", fourth
+    bullet: the workload includes causal forward passes.
+No formula is printed on any page. Readings taken (each listed in the design doc):
+  * attention is softmax(scale * Q K^T + mask) V, per query head h over key/value head
+    g = h // (Hq / Hkv) (grouped-query heads, contiguous groups);
+  * the causal mask is bottom-right aligned: query i sees key j iff j <= i + (Sk - Sq);
+  * a query row that sees no key has O = 0 and lse = -inf;
+  * lse is the natural log of sum_j exp(x_j) over the visible scaled scores x_j;
+  * the backward differentiates O only (not lse), using the softmax Jacobian diag(P) - P P^T;
+  * the monoid is the textbook online-softmax triple (m, l, o) with o unnormalised and the merge
+    (m,l,o) (+) (m',l',o') = (M, l e^{m-M} + l' e^{m'-M}, o e^{m-M} + o' e^{m'-M}), M = max(m, m'),
+    identity (-inf, 0, 0), and e^{-inf - M} taken as 0 so no inf - inf is ever formed.
+
+Layouts (row-major): Q, O, dO, dQ are [B, Sq, Hq, D]; K, V, dK, dV are [B, Sk, Hkv, D]; lse is
+[B, Hq, Sq]. Decode: q [N, Hq, D], packed k, v [T, Hkv, D], offsets [N + 1].
+
+The attention functions use the explicit two-pass softmax (pass 1: the row max; pass 2: the
+exponentials, their sum and the weighted sum of V). The monoid functions exist for the algebra
+tests only; the attention oracle does not use them.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+NEG_INF = -np.inf
+
+
+def _f64(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64)
+
+
+def _dims(q: np.ndarray, k: np.ndarray, v: np.ndarray):
+    if q.ndim != 4 or k.ndim != 4 or v.ndim != 4:
+        raise ValueError("q, k, v must be 4-D [B, S, H, D]")
+    B, Sq, Hq, D = q.shape
+    Bk, Sk, Hkv, Dk = k.shape
+    if Bk != B or Dk != D or v.shape[:3] != k.shape[:3]:
+        raise ValueError(f"shape mismatch q{q.shape} k{k.shape} v{v.shape}")
+    if Hkv <= 0 or Hq % Hkv != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    return B, Sq, Sk, Hq, Hkv, D, Hq // Hkv
+
+
+def visible_mask(Sq: int, Sk: int, causal: bool) -> np.ndarray:
+    """bool [Sq, Sk]: True where query i may attend to key j.
+
+    Causal masking (the "causal forward passes" of the aibriefing page, "Details") is read as
+    bottom-right aligned: j <= i + (Sk - Sq). With Sq == Sk this is the usual j <= i.
+    """
+    if not causal:
+        return np.ones((Sq, Sk), dtype=bool)
+    i = np.arange(Sq)[:, None]
+    j = np.arange(Sk)[None, :]
+    return j <= i + (Sk - Sq)
+
+
+def attention_scores(q, k, causal: bool, scale: float) -> np.ndarray:
+    """Scaled scores x[b, h, i, j] = scale * sum_d Q[b,i,h,d] K[b,j,h//G,d]; masked entries -inf.
+
+    The body of the attention comprehension ("Não escreva kernels, derive-os", "Aprofundamento",
+    first paragraph). Returns fp64 [B, Hq, Sq, Sk]; meant for small shapes.
+    """
+    q, k = _f64(q), _f64(k)
+    B, Sq, Sk, Hq, Hkv, D, G = _dims(q, k, k)
+    vis = visible_mask(Sq, Sk, causal)
+    x = np.empty((B, Hq, Sq, Sk), dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            xh = scale * (q[b, :, h, :] @ k[b, :, g, :].T)
+            x[b, h] = np.where(vis, xh, NEG_INF)
+    return x
+
+
+def _two_pass_softmax(x: np.ndarray, vis: np.ndarray):
+    """Explicit two-pass softmax of one head's score matrix x [Sq, Sk] under mask vis.
+
+    Pass 1 takes the row max M; pass 2 forms e^{x - M}, its sum Z and P = e / Z. Rows with no
+    visible key give P = 0, M = -inf, Z = 0. Returns (P, M, Z).
+    """
+    x = np.where(vis, x, NEG_INF)
+    has_key = vis.any(axis=1)
+    M = np.where(has_key, x.max(axis=1, initial=NEG_INF), NEG_INF)      # pass 1
+    M_safe = np.where(has_key, M, 0.0)
+    e = np.where(vis, np.exp(x - M_safe[:, None]), 0.0)                 # pass 2
+    Z = e.sum(axis=1)
+    Z_safe = np.where(Z > 0, Z, 1.0)
+    P = e / Z_safe[:, None]
+    return P, M, Z
+
+
+def attention_probs(q, k, causal: bool, scale: float) -> np.ndarray:
+    """Softmax probabilities P[b, h, i, j] (fp64), rows over visible keys; for invariant tests."""
+    q, k = _f64(q), _f64(k)
+    B, Sq, Sk, Hq, Hkv, D, G = _dims(q, k, k)
+    vis = visible_mask(Sq, Sk, causal)
+    x = attention_scores(q, k, causal, scale)
+    P = np.empty_like(x)
+    for b in range(B):
+        for h in range(Hq):
+            P[b, h] = _two_pass_softmax(x[b, h], vis)[0]
+    return P
+
+
+def attention_fwd(q, k, v, causal: bool, scale: float):
+    """Forward attention O = softmax(scale * Q K^T + mask) V and lse = M + ln Z, in fp64.
+
+    The plain definition that the flash form reaches up to rounding ("Não escreva kernels,
+    derive-os", "Aprofundamento", first paragraph). Returns (O [B,Sq,Hq,D], lse [B,Hq,Sq]).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Sq, Sk, Hq, Hkv, D, G = _dims(q, k, v)
+    vis = visible_mask(Sq, Sk, causal)
+    o = np.zeros((B, Sq, Hq, v.shape[3]), dtype=np.float64)
+    lse = np.full((B, Hq, Sq), NEG_INF, dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            x = scale * (q[b, :, h, :] @ k[b, :, g, :].T)
+            P, M, Z = _two_pass_softmax(x, vis)
+            o[b, :, h, :] = P @ v[b, :, g, :]
+            with np.errstate(divide="ignore"):
+                lse[b, h] = np.where(Z > 0, M + np.log(np.where(Z > 0, Z, 1.0)), NEG_INF)
+    return o, lse
+
+
+def attention_fwd_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows):
+    """Forward attention for selected query rows of one (batch, head): exact over all visible keys.
+
+    Same definition as ``attention_fwd``; used where the full output is too large for the oracle
+    (the 44k-token causal prefill of "Não escreva kernels, derive-os", "Aprofundamento", third
+    paragraph). Returns (O [len(rows), D], lse [len(rows)]).
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    g = h // G
+    kg = _f64(k[b, :, g, :])
+    vg = _f64(v[b, :, g, :])
+    qr = _f64(q[b, rows, h, :])
+    x = scale * (qr @ kg.T)                                     # [R, Sk]
+    if causal:
+        vis = np.arange(Sk)[None, :] <= (rows[:, None] + (Sk - Sq))
+    else:
+        vis = np.ones_like(x, dtype=bool)
+    P, M, Z = _two_pass_softmax(x, vis)
+    o = P @ vg
+    with np.errstate(divide="ignore"):
+        lse = np.where(Z > 0, M + np.log(np.where(Z > 0, Z, 1.0)), NEG_INF)
+    return o, lse
+
+
+def attention_bwd(q, k, v, do, causal: bool, scale: float):
+    """Backward of O = softmax(x) V with x = scale * Q K^T + mask, from the softmax Jacobian.
+
+    With P the softmax rows, dP = dO V^T and Delta_i = sum_d dO_i O_i = sum_j P_ij dP_ij, the
+    Jacobian diag(P) - P P^T gives dS_ij = P_ij (dP_ij - Delta_i); then
+    dQ = scale dS K, dK = scale dS^T Q and dV = P^T dO, dK and dV summed over the query heads that
+    share a key/value head. The backward "comes out of rewrites" of the same graph
+    ("Não escreva kernels, derive-os", "Perguntas frequentes", "O que o Tang propõe de diferente?").
+    O is recomputed here from the definition; lse is not differentiated.
+    Returns (dQ [B,Sq,Hq,D], dK [B,Sk,Hkv,D], dV [B,Sk,Hkv,D]).
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, Sq, Sk, Hq, Hkv, D, G = _dims(q, k, v)
+    if do.shape != q.shape:
+        raise ValueError("dO must have the shape of Q")
+    vis = visible_mask(Sq, Sk, causal)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            x = scale * (q[b, :, h, :] @ k[b, :, g, :].T)
+            P, _, _ = _two_pass_softmax(x, vis)
+            O = P @ v[b, :, g, :]
+            dP = do[b, :, h, :] @ v[b, :, g, :].T
+            delta = np.sum(do[b, :, h, :] * O, axis=1)
+            dS = P * (dP - delta[:, None])
+            dq[b, :, h, :] = scale * (dS @ k[b, :, g, :])
+            dk[b, :, g, :] += scale * (dS.T @ q[b, :, h, :])
+            dv[b, :, g, :] += P.T @ do[b, :, h, :]
+    return dq, dk, dv
+
+
+def decode_attention(q, k, v, offsets, scale: float):
+    """Decode attention: stream n's single query attends all L_n = off[n+1] - off[n] of its keys.
+
+    The decode streams of "Não escreva kernels, derive-os" ("Aprofundamento", third paragraph: 16 to
+    48 concurrent streams). The newest position sees every cached key, so there is no mask; this is
+    the forward with Sq = 1 and Sk = L_n. Splitting the keys and merging partial triples changes
+    only rounding, so the oracle does not split. A stream with no key gives O = 0, lse = -inf.
+    q [N, Hq, D]; packed k, v [T, Hkv, D]; offsets [N + 1]. Returns (O [N,Hq,D], lse [N,Hq]).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    off = np.asarray(offsets, dtype=np.int64)
+    N, Hq, D = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    o = np.zeros((N, Hq, D), dtype=np.float64)
+    lse = np.full((N, Hq), NEG_INF, dtype=np.float64)
+    for n in range(N):
+        s, e = int(off[n]), int(off[n + 1])
+        if e <= s:
+            continue
+        for h in range(Hq):
+            g = h // G
+            x = scale * (k[s:e, g, :] @ q[n, h, :])           # [L]
+            M = x.max()                                       # pass 1
+            w = np.exp(x - M)                                 # pass 2
+            Z = w.sum()
+            o[n, h, :] = (w / Z) @ v[s:e, g, :]
+            lse[n, h] = M + math.log(Z)
+    return o, lse
+
+
+# ---------------------------------------------------------------------------------------------
+# The online-softmax monoid, written out for the algebra tests ("Não escreva kernels, derive-os",
+# "Aprofundamento", first paragraph: the online softmax recognised as a monoid). A triple is
+# (m, l, o): running max, running sum of e^{x - m}, and the unnormalised accumulator sum e^{x-m} v.
+# ---------------------------------------------------------------------------------------------
+
+def monoid_identity(D: int):
+    """Identity triple (-inf, 0, 0)."""
+    return (NEG_INF, 0.0, np.zeros(D, dtype=np.float64))
+
+
+def monoid_leaf(x: float, v) -> tuple:
+    """Triple of one key with scaled score x and value row v: (x, 1, v)."""
+    return (float(x), 1.0, _f64(v).copy())
+
+
+def _weight(m: float, M: float) -> float:
+    # e^{m - M}, with e^{-inf - M} := 0 (also when M = -inf), so no inf - inf is formed.
+    if m == NEG_INF:
+        return 0.0
+    return math.exp(m - M)
+
+
+def monoid_merge(a: tuple, b: tuple) -> tuple:
+    """(m,l,o) (+) (m',l',o') = (M, l e^{m-M} + l' e^{m'-M}, o e^{m-M} + o' e^{m'-M}), M = max."""
+    m1, l1, o1 = a
+    m2, l2, o2 = b
+    M = max(m1, m2)
+    w1 = _weight(m1, M)
+    w2 = _weight(m2, M)
+    return (M, l1 * w1 + l2 * w2, _f64(o1) * w1 + _f64(o2) * w2)
+
+
+def monoid_finalize(t: tuple):
+    """Finalise a triple to (O = o / l, lse = m + ln l); the identity gives (0, -inf)."""
+    m, l, o = t
+    if l == 0.0:
+        return np.zeros_like(_f64(o)), NEG_INF
+    return _f64(o) / l, m + math.log(l)

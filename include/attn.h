@@ -1,0 +1,162 @@
+/*
+ * attn.h -- C ABI of libattn.so: online-softmax attention on NVIDIA B200 (sm_100a).
+ *
+ * What is computed. Scaled-dot-product attention written as one reduction over the keys under the
+ * online-softmax monoid (running max m, running sum l, rescaled accumulator o, with an associative
+ * merge): the form that "Não escreva kernels, derive-os" (ceviu.com.br, section "Aprofundamento",
+ * first paragraph) says flash attention falls out of once the online softmax is seen as a monoid.
+ * The backward is the gradient of the same expression (same page, "Perguntas frequentes",
+ * "O que o Tang propõe de diferente?"); causal forward passes are named on the aibriefing page
+ * "Tang Project Derives GPU Kernels via IR ..." ("Details"); the decode streams (16 to 48) and the
+ * 44k-token prefill are in the third paragraph of "Aprofundamento".
+ *
+ *   x_ij  = scale * sum_d Q[b,i,h,d] * K[b,j,g,d],  g = h / (Hq/Hkv)     (grouped-query heads)
+ *   causal: key j is visible to query i iff j <= i + (Sk - Sq)           (bottom-right aligned)
+ *   O[b,i,h,:] = sum_j softmax_j(x_i.) V[b,j,g,:],  lse[b,h,i] = ln sum_j exp(x_ij)  (natural log)
+ *   A query row that sees no key gets O = 0 and lse = -inf.
+ *
+ * Layouts (row-major, contiguous, no padding):
+ *   Q, O, dO, dQ : [B, Sq, Hq, D]      K, V, dK, dV : [B, Sk, Hkv, D]      lse : [B, Hq, Sq] fp32
+ *   decode: q, o : [N, Hq, D]   k, v : [T, Hkv, D] packed by stream   kv_offsets : [N+1] int32
+ * bf16 tensors are passed as void* to 16-bit storage (bfloat16 bit patterns); fp32 as float*.
+ *
+ * Conventions shared by every call:
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller. The library never allocates,
+ *     never frees and never synchronises (attn_get_device_status is the one call that waits).
+ *   - All work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream) in
+ *     stream order. Results are valid once that stream's prior work has completed.
+ *   - Arguments are validated on the host BEFORE anything is launched; on error nothing is
+ *     enqueued and an attn_status_t error code is returned. Checks: null pointers, B/H/S/D <= 0,
+ *     Hq % Hkv != 0, unsupported D, pointers not 16-byte aligned, workspace too small, device not
+ *     sm_100. Launch failures (cudaGetLastError after the launch) return ATTN_ERR_LAUNCH.
+ *   - Kernels that wait on on-chip barriers bound every wait; if a bound is hit the kernel records
+ *     ATTN_ERR_TIMEOUT in a device status word and exits (read it with attn_get_device_status).
+ *   - `scale` is used exactly as given (no default inside the ABI).
+ */
+#ifndef ATTN_H_
+#define ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, Hq % Hkv != 0, bad causal flag */
+  ATTN_ERR_UNSUPPORTED = 2,   /* head dim not supported by this entry point, or GPU not sm_100  */
+  ATTN_ERR_ALIGNMENT = 3,     /* a pointer is not 16-byte aligned                                */
+  ATTN_ERR_WORKSPACE = 4,     /* workspace pointer null or workspace_bytes too small             */
+  ATTN_ERR_LAUNCH = 5,        /* a CUDA launch failed                                            */
+  ATTN_ERR_TIMEOUT = 6        /* a kernel's bounded on-chip wait ran out (device status only)    */
+} attn_status_t;
+
+/* A cudaStream_t, passed as an opaque pointer so that this header needs no CUDA include. */
+typedef void* attn_stream_t;
+
+/* ------------------------------------------------------------------------------------------ *
+ * Forward.  ("Não escreva kernels, derive-os", "Aprofundamento", first paragraph: attention as
+ * one comprehension reduced under the online-softmax monoid.)
+ *
+ * attn_fwd: bf16 Q, K, V -> bf16 O and fp32 lse, fp32 accumulation on the tensor cores.
+ *   q [B,Sq,Hq,D] bf16, k/v [B,Sk,Hkv,D] bf16 (inputs, read only); o [B,Sq,Hq,D] bf16 and
+ *   lse [B,Hq,Sq] fp32 (outputs, fully overwritten; lse is required). D must be 64 or 128
+ *   (else ATTN_ERR_UNSUPPORTED). causal is 0 or 1.
+ * attn_fwd_f32: the same with fp32 tensors everywhere and genuine fp32 arithmetic (no TF32),
+ *   any D in [1, 256].
+ * ------------------------------------------------------------------------------------------ */
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                       int B, int Hq, int Hkv, int Sq, int Sk, int D, int causal, float scale,
+                       attn_stream_t stream);
+
+attn_status_t attn_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
+                           int B, int Hq, int Hkv, int Sq, int Sk, int D, int causal, float scale,
+                           attn_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------ *
+ * Backward.  (Same page, "Perguntas frequentes", "O que o Tang propõe de diferente?": the backward
+ * comes out of rewrites of the forward graph; the third paragraph of "Aprofundamento" notes a fused
+ * bf16 backward that misses an fp32 tolerance, so the bf16 path is held to bf16 tolerances.)
+ *
+ * With P = softmax rows recomputed from (Q, K, lse), dP = dO V^T, Delta_i = sum_d dO_i O_i and
+ * dS = P * (dP - Delta):  dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO, with dK and dV summed
+ * over the Hq/Hkv query heads that share a key/value head. Only O is differentiated (not lse).
+ *
+ * attn_bwd: bf16 q, k, v, o, dout and fp32 lse (as written by attn_fwd) -> bf16 dq, dk, dv (fully
+ *   overwritten). D must be 64 or 128. `workspace` is caller-owned device scratch of at least
+ *   attn_bwd_workspace_size(...) bytes, 256-byte aligned; its contents on entry do not matter and
+ *   it must not be used by other work on other streams while the call runs.
+ * attn_bwd_f32: fp32 everywhere, genuine fp32 arithmetic, any D in [1, 256]; its workspace size
+ *   is attn_bwd_f32_workspace_size(...).
+ * ------------------------------------------------------------------------------------------ */
+size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int D);
+
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                       const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                       void* workspace, size_t workspace_bytes,
+                       int B, int Hq, int Hkv, int Sq, int Sk, int D, int causal, float scale,
+                       attn_stream_t stream);
+
+size_t attn_bwd_f32_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int D);
+
+attn_status_t attn_bwd_f32(const float* q, const float* k, const float* v, const float* o,
+                           const float* lse, const float* dout, float* dq, float* dk, float* dv,
+                           void* workspace, size_t workspace_bytes,
+                           int B, int Hq, int Hkv, int Sq, int Sk, int D, int causal, float scale,
+                           attn_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------ *
+ * Split-KV decode.  (Decode streams of "Não escreva kernels, derive-os", "Aprofundamento", third
+ * paragraph; the aibriefing page, "Details", ties its 48-stream accuracy to split granularity.)
+ *
+ * Stream n has one query token q[n,:,:] and the L_n = kv_offsets[n+1] - kv_offsets[n] keys and
+ * values k/v[kv_offsets[n] : kv_offsets[n+1], :, :]; it attends to all of them (no mask). The keys
+ * of each (stream, kv head) are cut into C_n contiguous chunks of ceil(L_n / C_n) keys; each chunk
+ * yields a partial (m, l, o) triple in `workspace`, and a combine kernel merges the C_n triples with
+ * the monoid (m,l,o)+(m',l',o') = (M, l e^{m-M} + l' e^{m'-M}, o e^{m-M} + o' e^{m'-M}).
+ *
+ *   q [N,Hq,D] bf16; k, v [T,Hkv,D] bf16 with T = kv_offsets[N]; kv_offsets [N+1] int32 DEVICE
+ *   array, non-decreasing, kv_offsets[0] = 0 (not checked on the host: it lives on the device).
+ *   num_splits: [N] int32 DEVICE array of per-stream chunk counts, or NULL for the built-in rule
+ *   C(L) = min(max_splits, clamp(ceil(L/256), 4, 16)) (see attn_decode_default_splits); values
+ *   outside [1, max_splits] are clamped on the device. max_splits in [1, 64].
+ *   o [N,Hq,D] bf16 (output); lse [N,Hq] fp32 (output, may be NULL). A stream with L_n = 0 gets
+ *   O = 0 and lse = -inf. D must be 64 or 128.
+ *   workspace: caller-owned device scratch of at least attn_decode_workspace_size(N,Hq,D,max_splits)
+ *   bytes, 256-byte aligned (partial triples, fp32).
+ * ------------------------------------------------------------------------------------------ */
+size_t attn_decode_workspace_size(int N, int Hq, int D, int max_splits);
+
+attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v,
+                                  const int* kv_offsets, const int* num_splits, int max_splits,
+                                  void* o, float* lse, int N, int Hq, int Hkv, int D, float scale,
+                                  void* workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/* Host helper: the built-in split count for a stream of L keys (the rule named above). */
+int attn_decode_default_splits(int L, int max_splits);
+
+/* ------------------------------------------------------------------------------------------ *
+ * Status and introspection.
+ * ------------------------------------------------------------------------------------------ */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* attn_status_string(attn_status_t status);
+
+/* Waits for `stream`, then reads and clears the library's device status word on the current
+ * device: ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel gave up a bounded wait since the last read. */
+attn_status_t attn_get_device_status(attn_stream_t stream);
+
+/* Number of CUDA kernels this library has launched in this process (all devices, all calls). */
+uint64_t attn_launch_count(void);
+
+/* Name of the kernel family the last successful call of each kind dispatched to on this thread,
+ * e.g. "fwd_sm100_tcgen05" (static string). kind: 0 = forward, 1 = backward, 2 = decode. */
+const char* attn_last_path(int kind);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* ATTN_H_ */

@@ -1,0 +1,197 @@
+"""ctypes binding over libattn.so: argument marshalling only.
+
+torch is used here for device memory (output and workspace tensors) and for the current CUDA
+stream; every step of the computation runs in the library's CUDA kernels. If the shared library has
+not been built, the first call raises -- there is no other code path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
+
+STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_ALIGNMENT",
+          4: "ATTN_ERR_WORKSPACE", 5: "ATTN_ERR_LAUNCH", 6: "ATTN_ERR_TIMEOUT"}
+
+# (name, restype, argtypes) for every symbol include/attn.h declares
+_P, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_DIMS = [_I] * 6 + [_I, _F, _P]  # B, Hq, Hkv, Sq, Sk, D, causal, scale, stream
+SIGNATURES = [
+    ("attn_fwd", _I, [_P] * 5 + _DIMS),
+    ("attn_fwd_f32", _I, [_P] * 5 + _DIMS),
+    ("attn_bwd_workspace_size", _S, [_I] * 6),
+    ("attn_bwd", _I, [_P] * 9 + [_P, _S] + _DIMS),
+    ("attn_bwd_f32_workspace_size", _S, [_I] * 6),
+    ("attn_bwd_f32", _I, [_P] * 9 + [_P, _S] + _DIMS),
+    ("attn_decode_workspace_size", _S, [_I] * 4),
+    ("attn_decode_splitkv", _I, [_P] * 5 + [_I] + [_P, _P] + [_I] * 4 + [_F, _P, _S, _P]),
+    ("attn_decode_default_splits", _I, [_I, _I]),
+    ("attn_status_string", ctypes.c_char_p, [_I]),
+    ("attn_get_device_status", _I, [_P]),
+    ("attn_launch_count", ctypes.c_uint64, []),
+    ("attn_last_path", ctypes.c_char_p, [_I]),
+]
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libattn.so (once) and declare its C signatures."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libattn.so is not built ({LIB_PATH}); run "
+                              f"`python -m online_softmax_attention_fwd_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, res, args in SIGNATURES:
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().attn_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise AttnError(fn, status)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _expect(t: torch.Tensor, name: str, dtype, ndim: int):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-D tensor")
+
+
+def _prefill_dims(q, k, v):
+    B, Sq, Hq, D = q.shape
+    Bk, Sk, Hkv, Dk = k.shape
+    if Bk != B or Dk != D or tuple(v.shape) != tuple(k.shape):
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
+    return B, Hq, Hkv, Sq, Sk, D
+
+
+def _fwd(fn, dtype, q, k, v, causal, scale, out, lse):
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _expect(t, n, dtype, 4)
+    B, Hq, Hkv, Sq, Sk, D = _prefill_dims(q, k, v)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(fn, getattr(lib(), fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Sk, D,
+                                  int(bool(causal)), scale, _stream()))
+    return o, lse
+
+
+def fwd(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, lse=None):
+    """bf16 forward: (O [B,Sq,Hq,D] bf16, lse [B,Hq,Sq] fp32) via attn_fwd (tcgen05 kernel)."""
+    return _fwd("attn_fwd", torch.bfloat16, q, k, v, causal, scale, out, lse)
+
+
+def fwd_f32(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, lse=None):
+    """fp32 forward via attn_fwd_f32 (CUDA-core fp32 kernel, no TF32)."""
+    return _fwd("attn_fwd_f32", torch.float32, q, k, v, causal, scale, out, lse)
+
+
+def _bwd(fn, wsfn, dtype, q, k, v, o, lse, do, causal, scale, workspace):
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", do)):
+        _expect(t, n, dtype, 4)
+    _expect(lse, "lse", torch.float32, 3)
+    B, Hq, Hkv, Sq, Sk, D = _prefill_dims(q, k, v)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    need = getattr(lib(), wsfn)(B, Hq, Hkv, Sq, Sk, D)
+    if workspace is None:
+        workspace = torch.empty(max(int(need), 256), dtype=torch.uint8, device=q.device)
+    _check(fn, getattr(lib(), fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+                                  _ptr(dv), _ptr(workspace), workspace.numel(), B, Hq, Hkv, Sq, Sk, D,
+                                  int(bool(causal)), scale, _stream()))
+    return dq, dk, dv
+
+
+def bwd(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None, workspace=None):
+    """bf16 backward via attn_bwd: returns (dQ, dK, dV) bf16."""
+    return _bwd("attn_bwd", "attn_bwd_workspace_size", torch.bfloat16, q, k, v, o, lse, do, causal, scale,
+                workspace)
+
+
+def bwd_f32(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None, workspace=None):
+    """fp32 backward via attn_bwd_f32: returns (dQ, dK, dV) fp32."""
+    return _bwd("attn_bwd_f32", "attn_bwd_f32_workspace_size", torch.float32, q, k, v, o, lse, do, causal,
+                scale, workspace)
+
+
+def bwd_workspace_size(B, Hq, Hkv, Sq, Sk, D) -> int:
+    return int(lib().attn_bwd_workspace_size(B, Hq, Hkv, Sq, Sk, D))
+
+
+def decode_workspace_size(N, Hq, D, max_splits) -> int:
+    return int(lib().attn_decode_workspace_size(N, Hq, D, max_splits))
+
+
+def default_splits(L: int, max_splits: int = 16) -> int:
+    return int(lib().attn_decode_default_splits(int(L), int(max_splits)))
+
+
+def decode(q, k, v, kv_offsets, num_splits=None, max_splits: int = 16, scale: Optional[float] = None,
+           want_lse: bool = True, out=None, lse=None, workspace=None):
+    """Split-KV decode via attn_decode_splitkv: returns (O [N,Hq,D] bf16, lse [N,Hq] fp32 or None)."""
+    _expect(q, "q", torch.bfloat16, 3)
+    _expect(k, "k", torch.bfloat16, 3)
+    _expect(v, "v", torch.bfloat16, 3)
+    _expect(kv_offsets, "kv_offsets", torch.int32, 1)
+    if num_splits is not None:
+        _expect(num_splits, "num_splits", torch.int32, 1)
+    N, Hq, D = q.shape
+    Hkv = k.shape[1]
+    if tuple(v.shape) != tuple(k.shape) or k.shape[2] != D or kv_offsets.numel() != N + 1:
+        raise ValueError("shape mismatch in decode arguments")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    if want_lse and lse is None:
+        lse = torch.empty((N, Hq), dtype=torch.float32, device=q.device)
+    need = decode_workspace_size(N, Hq, D, max_splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check("attn_decode_splitkv", lib().attn_decode_splitkv(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(kv_offsets), _ptr(num_splits), int(max_splits), _ptr(o),
+        _ptr(lse) if want_lse else None, N, Hq, Hkv, D, scale, _ptr(workspace), workspace.numel(), _stream()))
+    return o, (lse if want_lse else None)
+
+
+def device_status() -> int:
+    """Wait for the current stream, then read and clear the device status word (0 = ok)."""
+    return int(lib().attn_get_device_status(_stream()))
+
+
+def launch_count() -> int:
+    return int(lib().attn_launch_count())
+
+
+def last_path(kind: int) -> str:
+    return lib().attn_last_path(int(kind)).decode()

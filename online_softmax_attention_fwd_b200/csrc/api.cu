@@ -1,0 +1,238 @@
+// api.cu -- the extern "C" boundary of libattn.so (declared in include/attn.h).
+//
+// Host-side only: argument validation (before anything is launched), dispatch to the kernel
+// families, the device status word read by attn_get_device_status, and a launch counter. Nothing
+// here allocates device memory or synchronises, except attn_get_device_status.
+#include <atomic>
+#include <mutex>
+
+#include <cuda_runtime.h>
+
+#include "../../include/attn.h"
+#include "kernels.h"
+
+namespace attn {
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+thread_local const char* g_last_path[3] = {"none", "none", "none"};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mu;
+int g_dev_arch[kMaxDevices];        // 0 = unknown, else major*10 + minor
+int* g_dev_status[kMaxDevices];     // device address of the status word, per device
+
+}  // namespace
+
+__device__ int g_status_word = 0;
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+static int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return (dev >= 0 && dev < kMaxDevices) ? dev : -1;
+}
+
+int* device_status_ptr() {
+  const int dev = current_device();
+  if (dev < 0) return nullptr;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_dev_status[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    g_dev_status[dev] = static_cast<int*>(p);
+  }
+  return g_dev_status[dev];
+}
+
+static bool device_is_sm100() {
+  const int dev = current_device();
+  if (dev < 0) return false;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_dev_arch[dev]) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return false;
+    g_dev_arch[dev] = major * 10 + minor;
+  }
+  return g_dev_arch[dev] == 100;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static attn_status_t check_problem(const Problem& p) {
+  if (p.B <= 0 || p.Hq <= 0 || p.Hkv <= 0 || p.Sq <= 0 || p.Sk <= 0 || p.D <= 0) return ATTN_ERR_INVALID_ARG;
+  if (p.Hq % p.Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (p.causal != 0 && p.causal != 1) return ATTN_ERR_INVALID_ARG;
+  // every index stays inside 32-bit element counts per tensor row set; whole tensors may be larger
+  const long long qel = static_cast<long long>(p.B) * p.Sq * p.Hq * p.D;
+  const long long kel = static_cast<long long>(p.B) * p.Sk * p.Hkv * p.D;
+  if (qel >= (1ll << 40) || kel >= (1ll << 40)) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+template <typename... P>
+static attn_status_t check_ptrs(P... ptrs) {
+  const void* all[] = {static_cast<const void*>(ptrs)...};
+  for (const void* x : all)
+    if (!x) return ATTN_ERR_INVALID_ARG;
+  for (const void* x : all)
+    if (!aligned16(x)) return ATTN_ERR_ALIGNMENT;
+  return ATTN_OK;
+}
+
+static attn_status_t launch_status(cudaError_t e) { return e == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH; }
+
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" {
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                       int Sq, int Sk, int D, int causal, float scale, attn_stream_t stream) {
+  const Problem p{B, Hq, Hkv, Sq, Sk, D, causal, scale};
+  attn_status_t s = check_problem(p);
+  if (s != ATTN_OK) return s;
+  if ((s = check_ptrs(q, k, v, o, lse)) != ATTN_OK) return s;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!device_is_sm100()) return ATTN_ERR_UNSUPPORTED;
+  const cudaError_t e = launch_fwd_sm100(p, q, k, v, o, lse, static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess) g_last_path[0] = "fwd_sm100_tcgen05";
+  return launch_status(e);
+}
+
+attn_status_t attn_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int Hq,
+                           int Hkv, int Sq, int Sk, int D, int causal, float scale, attn_stream_t stream) {
+  const Problem p{B, Hq, Hkv, Sq, Sk, D, causal, scale};
+  attn_status_t s = check_problem(p);
+  if (s != ATTN_OK) return s;
+  if ((s = check_ptrs(q, k, v, o, lse)) != ATTN_OK) return s;
+  if (D > 256) return ATTN_ERR_UNSUPPORTED;
+  if (!device_is_sm100()) return ATTN_ERR_UNSUPPORTED;
+  const cudaError_t e = launch_fwd_simt_f32(p, q, k, v, o, lse, static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess) g_last_path[0] = "fwd_simt_f32";
+  return launch_status(e);
+}
+
+static size_t delta_bytes(int B, int Hq, int Sq) {
+  return (static_cast<size_t>(B) * Hq * Sq * sizeof(float) + 255) & ~static_cast<size_t>(255);
+}
+
+size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int D) {
+  (void)Hkv;
+  (void)Sk;
+  (void)D;
+  if (B <= 0 || Hq <= 0 || Sq <= 0) return 0;
+  return delta_bytes(B, Hq, Sq);
+}
+
+size_t attn_bwd_f32_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int D) {
+  (void)Hkv;
+  (void)Sk;
+  (void)D;
+  if (B <= 0 || Hq <= 0 || Sq <= 0) return 0;
+  return delta_bytes(B, Hq, Sq);
+}
+
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                       const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                       int B, int Hq, int Hkv, int Sq, int Sk, int D, int causal, float scale,
+                       attn_stream_t stream) {
+  const Problem p{B, Hq, Hkv, Sq, Sk, D, causal, scale};
+  attn_status_t s = check_problem(p);
+  if (s != ATTN_OK) return s;
+  if ((s = check_ptrs(q, k, v, o, lse, dout, dq, dk, dv)) != ATTN_OK) return s;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < attn_bwd_workspace_size(B, Hq, Hkv, Sq, Sk, D)) return ATTN_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_ALIGNMENT;
+  if (!device_is_sm100()) return ATTN_ERR_UNSUPPORTED;
+  const cudaError_t e = launch_bwd_simt_bf16(p, q, k, v, o, lse, dout, dq, dk, dv, static_cast<float*>(workspace),
+                                             static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess) g_last_path[1] = "bwd_simt_bf16";
+  return launch_status(e);
+}
+
+attn_status_t attn_bwd_f32(const float* q, const float* k, const float* v, const float* o, const float* lse,
+                           const float* dout, float* dq, float* dk, float* dv, void* workspace,
+                           size_t workspace_bytes, int B, int Hq, int Hkv, int Sq, int Sk, int D, int causal,
+                           float scale, attn_stream_t stream) {
+  const Problem p{B, Hq, Hkv, Sq, Sk, D, causal, scale};
+  attn_status_t s = check_problem(p);
+  if (s != ATTN_OK) return s;
+  if ((s = check_ptrs(q, k, v, o, lse, dout, dq, dk, dv)) != ATTN_OK) return s;
+  if (D > 256) return ATTN_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < attn_bwd_f32_workspace_size(B, Hq, Hkv, Sq, Sk, D))
+    return ATTN_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_ALIGNMENT;
+  if (!device_is_sm100()) return ATTN_ERR_UNSUPPORTED;
+  const cudaError_t e = launch_bwd_simt_f32(p, q, k, v, o, lse, dout, dq, dk, dv, static_cast<float*>(workspace),
+                                            static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess) g_last_path[1] = "bwd_simt_f32";
+  return launch_status(e);
+}
+
+size_t attn_decode_workspace_size(int N, int Hq, int D, int max_splits) {
+  if (N <= 0 || Hq <= 0 || D <= 0 || max_splits <= 0) return 0;
+  return decode_workspace_bytes(N, Hq, D, max_splits);
+}
+
+int attn_decode_default_splits(int L, int max_splits) {
+  if (max_splits <= 0) return 0;
+  return decode_default_splits(L < 0 ? 0 : L, max_splits);
+}
+
+attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, const int* kv_offsets,
+                                  const int* num_splits, int max_splits, void* o, float* lse, int N, int Hq,
+                                  int Hkv, int D, float scale, void* workspace, size_t workspace_bytes,
+                                  attn_stream_t stream) {
+  if (N <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (max_splits < 1 || max_splits > 64) return ATTN_ERR_INVALID_ARG;
+  if (N > 65535 || static_cast<long long>(N) * Hq >= (1ll << 31)) return ATTN_ERR_INVALID_ARG;
+  attn_status_t s = check_ptrs(q, k, v, kv_offsets, o);
+  if (s != ATTN_OK) return s;
+  if (num_splits && !aligned16(num_splits)) return ATTN_ERR_ALIGNMENT;
+  if (lse && !aligned16(lse)) return ATTN_ERR_ALIGNMENT;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < decode_workspace_bytes(N, Hq, D, max_splits)) return ATTN_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_ALIGNMENT;
+  if (!device_is_sm100()) return ATTN_ERR_UNSUPPORTED;
+  const DecodeProblem p{N, Hq, Hkv, D, max_splits, scale};
+  const cudaError_t e = launch_decode(p, q, k, v, kv_offsets, num_splits, o, lse, workspace,
+                                      static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess) g_last_path[2] = "decode_splitkv_simt";
+  return launch_status(e);
+}
+
+const char* attn_status_string(attn_status_t status) {
+  switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported (head dim or device)";
+    case ATTN_ERR_ALIGNMENT: return "pointer not aligned";
+    case ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    case ATTN_ERR_LAUNCH: return "kernel launch failed";
+    case ATTN_ERR_TIMEOUT: return "a bounded on-chip wait timed out";
+  }
+  return "unknown status";
+}
+
+attn_status_t attn_get_device_status(attn_stream_t stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_LAUNCH;
+  int value = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&value, g_status_word, sizeof(int)) != cudaSuccess) return ATTN_ERR_LAUNCH;
+  if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_LAUNCH;
+  return static_cast<attn_status_t>(value);
+}
+
+uint64_t attn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* attn_last_path(int kind) {
+  if (kind < 0 || kind > 2) return "none";
+  return g_last_path[kind];
+}
+
+}  // extern "C"

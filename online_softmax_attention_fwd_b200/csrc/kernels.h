@@ -1,0 +1,48 @@
+// kernels.h -- internal launcher interface between the C ABI (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace attn {
+
+struct Problem {
+  int B, Hq, Hkv, Sq, Sk, D;
+  int causal;
+  float scale;
+};
+
+// Counts one kernel launch (reported by attn_launch_count).
+void note_launch();
+// Device pointer of the library's status word on the current device (nullptr if unavailable).
+int* device_status_ptr();
+
+// simt.cu: CUDA-core kernels, any D in [1, 256].
+cudaError_t launch_fwd_simt_f32(const Problem& p, const float* q, const float* k, const float* v, float* o,
+                                float* lse, cudaStream_t st);
+cudaError_t launch_fwd_simt_bf16(const Problem& p, const void* q, const void* k, const void* v, void* o,
+                                 float* lse, cudaStream_t st);
+cudaError_t launch_bwd_simt_f32(const Problem& p, const float* q, const float* k, const float* v, const float* o,
+                                const float* lse, const float* dout, float* dq, float* dk, float* dv,
+                                float* delta, cudaStream_t st);
+cudaError_t launch_bwd_simt_bf16(const Problem& p, const void* q, const void* k, const void* v, const void* o,
+                                 const float* lse, const void* dout, void* dq, void* dk, void* dv, float* delta,
+                                 cudaStream_t st);
+
+// decode.cu: split-KV decode, D in {64, 128}.
+struct DecodeProblem {
+  int N, Hq, Hkv, D, max_splits;
+  float scale;
+};
+size_t decode_workspace_bytes(int N, int Hq, int D, int max_splits);
+int decode_default_splits(int L, int max_splits);
+cudaError_t launch_decode(const DecodeProblem& p, const void* q, const void* k, const void* v,
+                          const int* kv_offsets, const int* num_splits, void* o, float* lse, void* workspace,
+                          cudaStream_t st);
+
+// fwd_sm100.cu: tcgen05 / TMA forward, bf16, D in {64, 128}.
+cudaError_t launch_fwd_sm100(const Problem& p, const void* q, const void* k, const void* v, void* o, float* lse,
+                             cudaStream_t st);
+
+}  // namespace attn

@@ -1,0 +1,79 @@
+"""GPU split-KV decode parity: libattn.so (through its C ABI) vs the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import online_softmax_attention_fwd_b200 as attn
+import oracle
+from online_softmax_attention_fwd_b200 import workloads as W
+from tests._util import assert_lse, assert_o_bf16, np64, max_abs
+
+pytestmark = pytest.mark.gpu
+
+
+def run_decode(w, num_splits=None, max_splits=16, want_lse=True):
+    dev = torch.device("cuda")
+    q, k, v, off = (t.to(dev) for t in (w.q, w.k, w.v, w.offsets))
+    ns = None if num_splits is None else torch.as_tensor(num_splits, dtype=torch.int32, device=dev)
+    o, lse = attn.decode(q, k, v, off, num_splits=ns, max_splits=max_splits, scale=w.scale,
+                         want_lse=want_lse)
+    torch.cuda.synchronize()
+    assert attn.device_status() == 0
+    return np64(o), (None if lse is None else np64(lse))
+
+
+def ref(w):
+    return oracle.decode_attention(np64(w.q), np64(w.k), np64(w.v), w.offsets.numpy(), w.scale)
+
+
+def test_decode48():
+    w = W.decode48()
+    o, lse = run_decode(w)
+    assert attn.last_path(2).startswith("decode_splitkv")
+    o_ref, lse_ref = ref(w)
+    assert_o_bf16(o, o_ref)
+    assert_lse(lse, lse_ref)
+
+
+@pytest.mark.parametrize("lengths,Hq,Hkv,D", [
+    ([1, 2, 3, 0, 5, 1000, 257], 8, 2, 128),      # length-1 and empty streams, ragged chunks
+    ([4096, 1, 513], 32, 8, 128),
+    ([300, 7000, 64], 16, 1, 64),                 # G = 16 (several passes of heads per CTA)
+    ([100, 200], 6, 3, 64),                       # G = 2
+    ([129, 31], 3, 3, 128),                       # G = 1
+    ([2048] * 5, 64, 8, 128),                     # G = 8 at D = 128
+])
+def test_decode_shapes(lengths, Hq, Hkv, D):
+    w = W.random_decode(len(lengths), Hq, Hkv, D, lengths, seed=sum(lengths) + Hq)
+    o, lse = run_decode(w)
+    o_ref, lse_ref = ref(w)
+    assert_o_bf16(o, o_ref)
+    assert_lse(lse, lse_ref)
+
+
+def test_merge_order_only_changes_rounding():
+    # the same streams cut into different numbers of chunks give the same result up to rounding
+    w = W.random_decode(6, 8, 2, 128, [3000, 1500, 17, 4096, 1024, 2500], seed=11)
+    o_ref, lse_ref = ref(w)
+    outs = []
+    for ns in ([1] * 6, [16] * 6, [3, 7, 1, 13, 2, 9], [64] * 6):
+        o, lse = run_decode(w, num_splits=ns, max_splits=64)
+        assert_o_bf16(o, o_ref)
+        assert_lse(lse, lse_ref)
+        outs.append(o)
+    for o in outs[1:]:
+        assert max_abs(o, outs[0]) <= 2e-2
+
+
+def test_lse_optional():
+    w = W.random_decode(3, 8, 2, 64, [10, 500, 2000], seed=2)
+    o, lse = run_decode(w, want_lse=False)
+    assert lse is None
+    assert_o_bf16(o, ref(w)[0])
+
+
+def test_empty_stream_gives_zero_and_minus_inf():
+    w = W.random_decode(3, 4, 2, 128, [0, 5, 0], seed=4)
+    o, lse = run_decode(w)
+    assert np.all(o[0] == 0) and np.all(o[2] == 0)
+    assert np.all(np.isneginf(lse[0])) and np.all(np.isneginf(lse[2]))

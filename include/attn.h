@@ -151,6 +151,19 @@ attn_status_t attn_get_device_status(attn_stream_t stream);
 /* Number of CUDA kernels this library has launched in this process (all devices, all calls). */
 uint64_t attn_launch_count(void);
 
+/* Opt-in per-kernel timing (for benchmarks). Between attn_profile_start() and attn_profile_stop()
+ * every kernel this library launches is bracketed by two CUDA events recorded on its launch stream
+ * (events are created on first use and reused; no device memory is allocated). attn_profile_stop()
+ * waits for the recorded events and sums the elapsed time per kernel family; the sums are then read
+ * with attn_profile_entries / _name / _total_ms / _launches (index 0 .. entries-1). Not for use
+ * while a stream is being captured into a CUDA graph. */
+attn_status_t attn_profile_start(void);
+attn_status_t attn_profile_stop(void);
+int attn_profile_entries(void);
+const char* attn_profile_name(int i);
+double attn_profile_total_ms(int i);
+int attn_profile_launches(int i);
+
 /* Name of the kernel family the last successful call of each kind dispatched to on this thread,
  * e.g. "fwd_sm100_tcgen05" (static string). kind: 0 = forward, 1 = backward, 2 = decode. */
 const char* attn_last_path(int kind);

@@ -28,5 +28,7 @@ from ._binding import (  # noqa: F401
     last_path,
     launch_count,
     lib,
+    profile_start,
+    profile_stop,
     status_string,
 )

@@ -35,6 +35,12 @@ SIGNATURES = [
     ("attn_get_device_status", _I, [_P]),
     ("attn_launch_count", ctypes.c_uint64, []),
     ("attn_last_path", ctypes.c_char_p, [_I]),
+    ("attn_profile_start", _I, []),
+    ("attn_profile_stop", _I, []),
+    ("attn_profile_entries", _I, []),
+    ("attn_profile_name", ctypes.c_char_p, [_I]),
+    ("attn_profile_total_ms", ctypes.c_double, [_I]),
+    ("attn_profile_launches", _I, [_I]),
 ]
 
 _lib = None
@@ -118,13 +124,13 @@ def fwd_f32(q, k, v, causal: bool = False, scale: Optional[float] = None, out=No
     return _fwd("attn_fwd_f32", torch.float32, q, k, v, causal, scale, out, lse)
 
 
-def _bwd(fn, wsfn, dtype, q, k, v, o, lse, do, causal, scale, workspace):
+def _bwd(fn, wsfn, dtype, q, k, v, o, lse, do, causal, scale, workspace, out=None):
     for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", do)):
         _expect(t, n, dtype, 4)
     _expect(lse, "lse", torch.float32, 3)
     B, Hq, Hkv, Sq, Sk, D = _prefill_dims(q, k, v)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dq, dk, dv = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)) if out is None else out
     need = getattr(lib(), wsfn)(B, Hq, Hkv, Sq, Sk, D)
     if workspace is None:
         workspace = torch.empty(max(int(need), 256), dtype=torch.uint8, device=q.device)
@@ -134,16 +140,17 @@ def _bwd(fn, wsfn, dtype, q, k, v, o, lse, do, causal, scale, workspace):
     return dq, dk, dv
 
 
-def bwd(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None, workspace=None):
-    """bf16 backward via attn_bwd: returns (dQ, dK, dV) bf16."""
+def bwd(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None, workspace=None, out=None):
+    """bf16 backward via attn_bwd: returns (dQ, dK, dV) bf16 (written into `out` if given)."""
     return _bwd("attn_bwd", "attn_bwd_workspace_size", torch.bfloat16, q, k, v, o, lse, do, causal, scale,
-                workspace)
+                workspace, out)
 
 
-def bwd_f32(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None, workspace=None):
-    """fp32 backward via attn_bwd_f32: returns (dQ, dK, dV) fp32."""
+def bwd_f32(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None, workspace=None,
+            out=None):
+    """fp32 backward via attn_bwd_f32: returns (dQ, dK, dV) fp32 (written into `out` if given)."""
     return _bwd("attn_bwd_f32", "attn_bwd_f32_workspace_size", torch.float32, q, k, v, o, lse, do, causal,
-                scale, workspace)
+                scale, workspace, out)
 
 
 def bwd_workspace_size(B, Hq, Hkv, Sq, Sk, D) -> int:
@@ -195,3 +202,15 @@ def launch_count() -> int:
 
 def last_path(kind: int) -> str:
     return lib().attn_last_path(int(kind)).decode()
+
+
+def profile_start() -> None:
+    _check("attn_profile_start", lib().attn_profile_start())
+
+
+def profile_stop() -> dict:
+    """Stop the per-kernel profiler; returns {kernel family: (total ms, launches)}."""
+    _check("attn_profile_stop", lib().attn_profile_stop())
+    L = lib()
+    return {L.attn_profile_name(i).decode(): (float(L.attn_profile_total_ms(i)), int(L.attn_profile_launches(i)))
+            for i in range(L.attn_profile_entries())}

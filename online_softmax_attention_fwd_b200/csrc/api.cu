@@ -5,6 +5,8 @@
 // here allocates device memory or synchronises, except attn_get_device_status.
 #include <atomic>
 #include <mutex>
+#include <string.h>
+#include <vector>
 
 #include <cuda_runtime.h>
 
@@ -26,7 +28,54 @@ int* g_dev_status[kMaxDevices];     // device address of the status word, per de
 
 __device__ int g_status_word = 0;
 
-void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+// ---------------------------------------------------------------------------------------------
+// Opt-in per-kernel timing: while on, every launch is bracketed by two CUDA events recorded on its
+// stream; attn_profile_stop() waits for them and sums the elapsed time per kernel family.
+// ---------------------------------------------------------------------------------------------
+namespace {
+struct ProfRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+struct ProfSum {
+  const char* name;
+  double ms;
+  int launches;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof_recs;
+std::vector<cudaEvent_t> g_prof_pool;
+std::vector<ProfSum> g_prof_sums;
+
+cudaEvent_t prof_event() {
+  if (!g_prof_pool.empty()) {
+    cudaEvent_t e = g_prof_pool.back();
+    g_prof_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+}  // namespace
+
+LaunchScope::LaunchScope(const char* name, cudaStream_t st) : name_(name), st_(st), slot_(-1) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (!g_prof_on) return;
+  ProfRec r{name, prof_event(), prof_event()};
+  if (!r.a || !r.b) return;
+  cudaEventRecord(r.a, st);
+  slot_ = static_cast<int>(g_prof_recs.size());
+  g_prof_recs.push_back(r);
+}
+
+LaunchScope::~LaunchScope() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (slot_ < 0) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (slot_ < static_cast<int>(g_prof_recs.size())) cudaEventRecord(g_prof_recs[slot_].b, st_);
+}
 
 static int current_device() {
   int dev = -1;
@@ -229,6 +278,64 @@ attn_status_t attn_get_device_status(attn_stream_t stream) {
 }
 
 uint64_t attn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+attn_status_t attn_profile_start(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& r : g_prof_recs) {
+    g_prof_pool.push_back(r.a);
+    g_prof_pool.push_back(r.b);
+  }
+  g_prof_recs.clear();
+  g_prof_sums.clear();
+  g_prof_on = true;
+  return ATTN_OK;
+}
+
+attn_status_t attn_profile_stop(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = false;
+  g_prof_sums.clear();
+  attn_status_t st = ATTN_OK;
+  for (auto& r : g_prof_recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) {
+      st = ATTN_ERR_LAUNCH;
+      continue;
+    }
+    bool found = false;
+    for (auto& s : g_prof_sums)
+      if (strcmp(s.name, r.name) == 0) {
+        s.ms += ms;
+        s.launches += 1;
+        found = true;
+      }
+    if (!found) g_prof_sums.push_back(ProfSum{r.name, static_cast<double>(ms), 1});
+    g_prof_pool.push_back(r.a);
+    g_prof_pool.push_back(r.b);
+  }
+  g_prof_recs.clear();
+  return st;
+}
+
+int attn_profile_entries(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  return static_cast<int>(g_prof_sums.size());
+}
+
+const char* attn_profile_name(int i) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  return (i >= 0 && i < static_cast<int>(g_prof_sums.size())) ? g_prof_sums[i].name : "";
+}
+
+double attn_profile_total_ms(int i) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  return (i >= 0 && i < static_cast<int>(g_prof_sums.size())) ? g_prof_sums[i].ms : 0.0;
+}
+
+int attn_profile_launches(int i) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  return (i >= 0 && i < static_cast<int>(g_prof_sums.size())) ? g_prof_sums[i].launches : 0;
+}
 
 const char* attn_last_path(int kind) {
   if (kind < 0 || kind > 2) return "none";

@@ -295,10 +295,12 @@ cudaError_t launch_split(const DecodeProblem& p, const void* q, const void* k, c
                          cudaStream_t st) {
   const int npass = (p.Hq / p.Hkv) / GT;
   dim3 grid(p.max_splits, p.Hkv * npass, p.N);
-  decode_split_kernel<D, GT><<<grid, 128, 0, st>>>(
-      static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v), offsets,
-      num_splits, p.max_splits, p.Hq, p.Hkv, p.scale * kLog2e, part_o, part_ml);
-  note_launch();
+  {
+    LaunchScope ls("decode_split", st);
+    decode_split_kernel<D, GT><<<grid, 128, 0, st>>>(
+        static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v),
+        offsets, num_splits, p.max_splits, p.Hq, p.Hkv, p.scale * kLog2e, part_o, part_ml);
+  }
   return cudaGetLastError();
 }
 
@@ -329,9 +331,11 @@ cudaError_t launch_decode_d(const DecodeProblem& p, const void* q, const void* k
   }
   if (e != cudaSuccess) return e;
   const long long warps = static_cast<long long>(p.N) * p.Hq;
-  decode_combine_kernel<D><<<static_cast<unsigned>((warps + 3) / 4), 128, 0, st>>>(
-      part_o, part_ml, offsets, num_splits, p.max_splits, p.N, p.Hq, static_cast<uint16_t*>(o), lse);
-  note_launch();
+  {
+    LaunchScope ls("decode_combine", st);
+    decode_combine_kernel<D><<<static_cast<unsigned>((warps + 3) / 4), 128, 0, st>>>(
+        part_o, part_ml, offsets, num_splits, p.max_splits, p.N, p.Hq, static_cast<uint16_t*>(o), lse);
+  }
   return cudaGetLastError();
 }
 

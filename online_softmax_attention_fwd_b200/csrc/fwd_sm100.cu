@@ -403,8 +403,10 @@ cudaError_t launch_fwd_sm100_d(const Problem& p, const void* q, const void* k, c
   a.lse = lse;
   a.status = device_status_ptr();
   dim3 grid(a.n_qtiles, p.Hq, p.B);
-  fwd_sm100_kernel<D><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);
-  note_launch();
+  {
+    LaunchScope ls("fwd_sm100", st);
+    fwd_sm100_kernel<D><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);
+  }
   return cudaGetLastError();
 }
 

@@ -13,8 +13,18 @@ struct Problem {
   float scale;
 };
 
-// Counts one kernel launch (reported by attn_launch_count).
-void note_launch();
+// Brackets one kernel launch: counts it (attn_launch_count) and, while the opt-in profiler is on,
+// records CUDA events around it on the launch stream (attn_profile_*). `name` is a static string.
+class LaunchScope {
+ public:
+  LaunchScope(const char* name, cudaStream_t st);
+  ~LaunchScope();
+
+ private:
+  const char* name_;
+  cudaStream_t st_;
+  int slot_;
+};
 // Device pointer of the library's status word on the current device (nullptr if unavailable).
 int* device_status_ptr();
 

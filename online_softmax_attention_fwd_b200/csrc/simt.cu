@@ -281,10 +281,12 @@ template <typename T, int DPL>
 cudaError_t fwd_simt_dpl(const Problem& p, const void* q, const void* k, const void* v, void* o, float* lse,
                          cudaStream_t st) {
   const long long rows = static_cast<long long>(p.B) * p.Hq * p.Sq;
-  fwd_simt_kernel<T, DPL><<<blocks_for(rows), 128, 0, st>>>(
-      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), static_cast<T*>(o), lse, p.B,
-      p.Hq, p.Hkv, p.Sq, p.Sk, p.D, p.causal, p.scale);
-  note_launch();
+  {
+    LaunchScope ls(sizeof(T) == 4 ? "fwd_simt_f32" : "fwd_simt_bf16", st);
+    fwd_simt_kernel<T, DPL><<<blocks_for(rows), 128, 0, st>>>(
+        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), static_cast<T*>(o), lse, p.B,
+        p.Hq, p.Hkv, p.Sq, p.Sk, p.D, p.causal, p.scale);
+  }
   return cudaGetLastError();
 }
 
@@ -294,23 +296,29 @@ cudaError_t bwd_simt_dpl(const Problem& p, const void* q, const void* k, const v
                          cudaStream_t st) {
   const long long qrows = static_cast<long long>(p.B) * p.Hq * p.Sq;
   const long long krows = static_cast<long long>(p.B) * p.Hkv * p.Sk;
-  bwd_delta_kernel<T, DPL><<<blocks_for(qrows), 128, 0, st>>>(static_cast<const T*>(o),
-                                                               static_cast<const T*>(dout), delta, p.B, p.Hq,
-                                                               p.Sq, p.D);
-  note_launch();
+  {
+    LaunchScope ls("bwd_simt_delta", st);
+    bwd_delta_kernel<T, DPL><<<blocks_for(qrows), 128, 0, st>>>(static_cast<const T*>(o),
+                                                                 static_cast<const T*>(dout), delta, p.B, p.Hq,
+                                                                 p.Sq, p.D);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_dq_simt_kernel<T, DPL><<<blocks_for(qrows), 128, 0, st>>>(
-      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), static_cast<const T*>(dout),
-      lse, delta, static_cast<T*>(dq), p.B, p.Hq, p.Hkv, p.Sq, p.Sk, p.D, p.causal, p.scale);
-  note_launch();
+  {
+    LaunchScope ls("bwd_simt_dq", st);
+    bwd_dq_simt_kernel<T, DPL><<<blocks_for(qrows), 128, 0, st>>>(
+        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), static_cast<const T*>(dout),
+        lse, delta, static_cast<T*>(dq), p.B, p.Hq, p.Hkv, p.Sq, p.Sk, p.D, p.causal, p.scale);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_dkdv_simt_kernel<T, DPL><<<blocks_for(krows), 128, 0, st>>>(
-      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), static_cast<const T*>(dout),
-      lse, delta, static_cast<T*>(dk), static_cast<T*>(dv), p.B, p.Hq, p.Hkv, p.Sq, p.Sk, p.D, p.causal,
-      p.scale);
-  note_launch();
+  {
+    LaunchScope ls("bwd_simt_dkdv", st);
+    bwd_dkdv_simt_kernel<T, DPL><<<blocks_for(krows), 128, 0, st>>>(
+        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), static_cast<const T*>(dout),
+        lse, delta, static_cast<T*>(dk), static_cast<T*>(dv), p.B, p.Hq, p.Hkv, p.Sq, p.Sk, p.D, p.causal,
+        p.scale);
+  }
   return cudaGetLastError();
 }
 

@@ -134,6 +134,24 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v,
                                   void* o, float* lse, int N, int Hq, int Hkv, int D, float scale,
                                   void* workspace, size_t workspace_bytes, attn_stream_t stream);
 
+/* Split-KV decode that allocates nothing (the pages have no counterpart: this entry point exists
+ * for callers of this library that cannot hand it a workspace -- a host framework that owns all
+ * device memory through its own pool and gives plugins no scratch, or a latency-bound serving loop
+ * that may not call cudaMalloc, which can synchronise the device, on its hot path).
+ * Same arguments, kernels and results as attn_decode_splitkv, minus the workspace: the partial
+ * (m, l, o) triples live in a 16 MiB array compiled into the library, which every GPU that loads the
+ * library holds until the process exits. Problems needing more than 16 MiB of partial triples
+ * (attn_decode_workspace_size(N, Hq, D, max_splits) > 16777216) return ATTN_ERR_WORKSPACE before
+ * anything is launched; e.g. 48 streams x 32 heads x 16 splits at D = 128 need 12.8 MB and fit.
+ * The first call on each device looks up the array's device address (once per device, with that
+ * device current); make that first call before any stream capture. All calls share the array and
+ * leave their partial triples in it; nothing has to start at zero. Calls that overlap on the GPU
+ * (other streams or threads) race on the array and give wrong results: serialise them. */
+attn_status_t attn_decode_splitkv_static(const void* q, const void* k, const void* v,
+                                         const int* kv_offsets, const int* num_splits, int max_splits,
+                                         void* o, float* lse, int N, int Hq, int Hkv, int D,
+                                         float scale, attn_stream_t stream);
+
 /* Host helper: the built-in split count for a stream of L keys (the rule named above). */
 int attn_decode_default_splits(int L, int max_splits);
 

@@ -30,6 +30,7 @@ SIGNATURES = [
     ("attn_bwd_f32", _I, [_P] * 9 + [_P, _S] + _DIMS),
     ("attn_decode_workspace_size", _S, [_I] * 4),
     ("attn_decode_splitkv", _I, [_P] * 5 + [_I] + [_P, _P] + [_I] * 4 + [_F, _P, _S, _P]),
+    ("attn_decode_splitkv_static", _I, [_P] * 5 + [_I] + [_P, _P] + [_I] * 4 + [_F, _P]),
     ("attn_decode_default_splits", _I, [_I, _I]),
     ("attn_status_string", ctypes.c_char_p, [_I]),
     ("attn_get_device_status", _I, [_P]),

@@ -18,7 +18,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_PATH = os.path.join(HERE, "libattn.so")
-SOURCES = ["api.cu", "simt.cu", "decode.cu", "decode_static.cu", "fwd_sm100.cu"]
+SOURCES = ["api.cu", "simt.cu", "decode.cu", "decode_static.cu", "fwd_sm100.cu", "bwd_sm100.cu"]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ARCH_FLAGS + ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE,

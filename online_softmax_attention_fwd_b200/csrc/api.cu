@@ -173,9 +173,8 @@ static size_t delta_bytes(int B, int Hq, int Sq) {
 size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int D) {
   (void)Hkv;
   (void)Sk;
-  (void)D;
-  if (B <= 0 || Hq <= 0 || Sq <= 0) return 0;
-  return delta_bytes(B, Hq, Sq);
+  if (B <= 0 || Hq <= 0 || Sq <= 0 || D <= 0) return 0;
+  return bwd_sm100_workspace_bytes(B, Hq, Sq, D);
 }
 
 size_t attn_bwd_f32_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int D) {
@@ -198,9 +197,9 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
   if (!workspace || workspace_bytes < attn_bwd_workspace_size(B, Hq, Hkv, Sq, Sk, D)) return ATTN_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_ALIGNMENT;
   if (!device_is_sm100()) return ATTN_ERR_UNSUPPORTED;
-  const cudaError_t e = launch_bwd_simt_bf16(p, q, k, v, o, lse, dout, dq, dk, dv, static_cast<float*>(workspace),
-                                             static_cast<cudaStream_t>(stream));
-  if (e == cudaSuccess) g_last_path[1] = "bwd_simt_bf16";
+  const cudaError_t e = launch_bwd_sm100(p, q, k, v, o, lse, dout, dq, dk, dv, workspace,
+                                         static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess) g_last_path[1] = "bwd_sm100_tcgen05";
   return launch_status(e);
 }
 

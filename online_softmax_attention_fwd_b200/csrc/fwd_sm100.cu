@@ -25,6 +25,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tma_host.h"
 
 namespace attn {
 namespace {
@@ -96,8 +97,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = a.n_qtiles - 1 - static_cast<int>(blockIdx.x);  // longest causal tiles first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // blockIdx.y walks the query tiles from the last (longest under a causal mask) to the first, and
+  // blockIdx.x, which varies fastest in launch order, covers every (batch, head): the longest tiles
+  // of all heads start first.
+  const int tile = a.n_qtiles - 1 - static_cast<int>(blockIdx.y);
+  const int h = static_cast<int>(blockIdx.x) % a.Hq, b = static_cast<int>(blockIdx.x) / a.Hq;
   const int g = h / (a.Hq / a.Hkv);
   const int q0 = tile * kBM;
   int kv_end = a.Sk;  // keys [0, kv_end) can be visible to some row of this tile
@@ -345,48 +349,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------------------------
 // host side: tensor maps and launch
 // ---------------------------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// 4-D map over a [B, S, H, D] bf16 tensor: dims (D, H, S, B); box (64, 1, 128, 1), 128-byte swizzle.
-bool make_map_bshd(CUtensorMap* map, const void* base, int B, int S, int H, int D) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(S),
-                              static_cast<cuuint64_t>(B)};
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
-                                 static_cast<cuuint64_t>(S) * H * D * 2};
-  const cuuint32_t box[4] = {64, 1, 128, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <int D>
 cudaError_t launch_fwd_sm100_d(const Problem& p, const void* q, const void* k, const void* v, void* o, float* lse,
                                cudaStream_t st) {
   using C = FwdCfg<D>;
   CUtensorMap mq, mk, mv;
-  if (!make_map_bshd(&mq, q, p.B, p.Sq, p.Hq, D) || !make_map_bshd(&mk, k, p.B, p.Sk, p.Hkv, D) ||
-      !make_map_bshd(&mv, v, p.B, p.Sk, p.Hkv, D))
+  if (!make_map_bf16_sw128(&mq, q, p.B, p.Sq, p.Hq, D, kBM) || !make_map_bf16_sw128(&mk, k, p.B, p.Sk, p.Hkv, D, kBN) ||
+      !make_map_bf16_sw128(&mv, v, p.B, p.Sk, p.Hkv, D, kBN))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
@@ -402,7 +371,7 @@ cudaError_t launch_fwd_sm100_d(const Problem& p, const void* q, const void* k, c
   a.o = static_cast<uint16_t*>(o);
   a.lse = lse;
   a.status = device_status_ptr();
-  dim3 grid(a.n_qtiles, p.Hq, p.B);
+  dim3 grid(p.Hq * p.B, a.n_qtiles);
   {
     LaunchScope ls("fwd_sm100", st);
     fwd_sm100_kernel<D><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);

@@ -55,4 +55,11 @@ cudaError_t launch_decode(const DecodeProblem& p, const void* q, const void* k, 
 cudaError_t launch_fwd_sm100(const Problem& p, const void* q, const void* k, const void* v, void* o, float* lse,
                              cudaStream_t st);
 
+// bwd_sm100.cu: tcgen05 / TMA backward, bf16, D in {64, 128}; workspace = fp32 dQ accumulator
+// [B, Sq, Hq, D] + lse2 [B, Hq, Sq] + Delta [B, Hq, Sq], each 256-byte aligned.
+size_t bwd_sm100_workspace_bytes(int B, int Hq, int Sq, int D);
+cudaError_t launch_bwd_sm100(const Problem& p, const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                             cudaStream_t st);
+
 }  // namespace attn

@@ -10,7 +10,7 @@
 
 #include <cuda_runtime.h>
 
-#include "../../include/attn.h"
+#include "attn.h"
 #include "kernels.h"
 
 namespace attn {

@@ -198,8 +198,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t kIdS = idesc_bf16_f32(kBN, kBM, 0, 0);  // S^T, dP^T
       constexpr uint32_t kIdG = idesc_bf16_f32(kBN, D, 0, 1);    // dV, dK
       constexpr uint32_t kIdQ = idesc_bf16_f32(128, kBM, 1, 1);  // dQ^T (M = 128 also for D = 64)
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO);
-      const uint32_t aP = smem_u32(sP), aDS = smem_u32(sDS);
+      // base descriptors, built once; each MMA only moves the start address
+      const uint64_t kK = sdesc_sw128(smem_u32(sK), 16, 1024);        // K-major operands
+      const uint64_t kV = sdesc_sw128(smem_u32(sV), 16, 1024);
+      const uint64_t kQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t kDO = sdesc_sw128(smem_u32(sDO), 16, 1024);
+      const uint64_t kP = sdesc_sw128(smem_u32(sP), 16, 1024);
+      const uint64_t kDS = sdesc_sw128(smem_u32(sDS), 16, 1024);
+      const uint64_t mQ = sdesc_sw128(smem_u32(sQ), kQAtom, 1024);    // MN-major operands
+      const uint64_t mDO = sdesc_sw128(smem_u32(sDO), kQAtom, 1024);
+      const uint64_t mK = sdesc_sw128(smem_u32(sK), kKAtom, 1024);
+      const uint64_t mDS = sdesc_sw128(smem_u32(sDS), kQAtom, 1024);
       bool ok = mbar_wait(kv_full, 0, abort, a.status);
       for (int j = 0; ok && j <= n_it; ++j) {
         if (j < n_it) {
@@ -207,14 +216,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(q_full + s, (j / C::kStages) & 1, abort, a.status)) break;
           if (!mbar_wait(st_free, (j & 1) ^ 1, abort, a.status)) break;
           tc_fence_after();
-#pragma unroll 1
+          const uint64_t q = sdesc_advance(kQ, s * C::kQBytes), dO = sdesc_advance(kDO, s * C::kQBytes);
+#pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t ok_ = (kk >> 2) * kKAtom + (kk & 3) * 32;
             const uint32_t oq = (kk >> 2) * kQAtom + (kk & 3) * 32;
-            umma_ss(tmem + C::kColS, sdesc_sw128(aK + ok_, 16, 1024),
-                    sdesc_sw128(aQ + s * C::kQBytes + oq, 16, 1024), kIdS, kk > 0);
-            umma_ss(tmem + C::kColDP, sdesc_sw128(aV + ok_, 16, 1024),
-                    sdesc_sw128(aDO + s * C::kQBytes + oq, 16, 1024), kIdS, kk > 0);
+            umma_ss(tmem + C::kColS, sdesc_advance(kK, ok_), sdesc_advance(q, oq), kIdS, kk > 0);
+            umma_ss(tmem + C::kColDP, sdesc_advance(kV, ok_), sdesc_advance(dO, oq), kIdS, kk > 0);
           }
           umma_commit(s_full);
         }
@@ -224,23 +232,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(p_full, jj & 1, abort, a.status)) break;
           if (!mbar_wait(dq_free, (jj & 1) ^ 1, abort, a.status)) break;
           tc_fence_after();
+          const uint64_t q = sdesc_advance(mQ, s * C::kQBytes), dO = sdesc_advance(mDO, s * C::kQBytes);
           // dV += P^T dO, dK += dS^T Q: K = 64 query rows in 4 steps of 16
-#pragma unroll 1
+#pragma unroll
           for (int kk = 0; kk < kBM / 16; ++kk) {
             const uint32_t oa = kk * 32;          // 16 rows = 32 bytes along the swizzled K-major row
             const uint32_t ob = kk * 16 * 128;    // 16 rows of 128 bytes in the MN-major operand
             const uint32_t acc = (jj > 0 || kk > 0);
-            umma_ss(tmem + C::kColDV, sdesc_sw128(aP + oa, 16, 1024),
-                    sdesc_sw128(aDO + s * C::kQBytes + ob, kQAtom, 1024), kIdG, acc);
-            umma_ss(tmem + C::kColDK, sdesc_sw128(aDS + oa, 16, 1024),
-                    sdesc_sw128(aQ + s * C::kQBytes + ob, kQAtom, 1024), kIdG, acc);
+            umma_ss(tmem + C::kColDV, sdesc_advance(kP, oa), sdesc_advance(dO, ob), kIdG, acc);
+            umma_ss(tmem + C::kColDK, sdesc_advance(kDS, oa), sdesc_advance(q, ob), kIdG, acc);
           }
           // dQ^T = K^T dS^T: K = 128 keys in 8 steps of 16
-#pragma unroll 1
+#pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
             const uint32_t o = kk * 16 * 128;
-            umma_ss(tmem + C::kColDQ, sdesc_sw128(aK + o, kKAtom, 1024), sdesc_sw128(aDS + o, kQAtom, 1024), kIdQ,
-                    kk > 0);
+            umma_ss(tmem + C::kColDQ, sdesc_advance(mK, o), sdesc_advance(mDS, o), kIdQ, kk > 0);
           }
           umma_commit(q_empty + s);
           umma_commit(pds_free);

@@ -1,27 +1,31 @@
 // fwd_sm100.cu -- attention forward on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
 //
 // The forward is one reduction over key blocks under the online-softmax monoid ("Não escreva
-// kernels, derive-os", "Aprofundamento", first paragraph): for a tile of 128 query rows the CTA
-// keeps, per row, the triple (m, l, O) -- running max (base-2 units), running sum of 2^(s - m) and
-// the unnormalised output -- and folds in one 128-key block at a time:
+// kernels, derive-os", "Aprofundamento", first paragraph): for every query row the CTA keeps the
+// triple (m, l, O) -- running max (base-2 units), running sum of 2^(s - m) and the unnormalised
+// output -- and folds in one 64-key block at a time:
 //   S = Q K^T (tensor cores, fp32 in TMEM), m' = max(m, rowmax S), P = 2^(S - m'),
 //   l = l 2^(m - m') + rowsum P, O = O 2^(m - m') + P V (tensor cores, fp32 in TMEM).
 // The two contractions are dense, so they run as tcgen05.mma (bf16 operands from shared memory,
 // fp32 accumulators in tensor memory); the row statistics run on the CUDA cores, one thread per row.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax: read S from TMEM, mask, row max / sum, write P (bf16, swizzled) to SMEM,
-//              rescale O in TMEM when a row max grows by more than 2^8, epilogue O / l and lse.
-//   warp 4     TMA producer: Q tile once, then K and V blocks into a ring of stages.
-//   warp 5     TMEM allocator and MMA issuer (one thread): S_j = Q K_j^T into one of two S buffers,
-//              then O += P_{j-1} V_{j-1}, so the next S overlaps the softmax of the current block.
+// A CTA owns two 128-row query tiles of one head and streams the key/value blocks once for both,
+// which halves the K/V bytes each SM pulls from L2 per tensor-core FLOP (with one tile per CTA
+// the SM's L2 read bandwidth, not the tensor cores, set the pace). Warp roles (320 threads):
+//   warps 0-3 / 4-7  softmax of tile 0 / tile 1: read S from TMEM, mask, row max / sum, write P
+//                    (bf16, swizzled, double-buffered) to SMEM, rescale O in TMEM when a row max
+//                    grows by more than 2^8, epilogue O / l and lse. With two P buffers per tile the
+//                    softmax waits for a PV only when it must rescale O.
+//   warp 8           TMA producer: both Q tiles once, then K and V blocks through a ring.
+//   warp 9           TMEM allocator and MMA issuer (one thread): S of block j for both tiles
+//                    (double-buffered in TMEM), then P V of block j - 1 for both tiles, so that the
+//                    tensor cores work on one tile while the other tile's softmax runs.
 // Lazy rescaling: a row keeps its old max m while the block max stays within m + 8 (base 2); P then
 // stays <= 256 and the final O / l and lse = m + log2 l use the same m, so the result is exact.
 //
 // Shared-memory tiles use the 128-byte swizzle: Q, K and P are K-major (rows of 64 bf16 = 128 B),
 // V is read as an MN-major operand (its head dim is contiguous). Every wait is bounded (common.cuh).
 #include <math.h>
-#include <stdio.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -30,33 +34,36 @@
 namespace attn {
 namespace {
 
-constexpr int kBM = 128;  // query rows per tile
-constexpr int kBN = 128;  // keys per block
-constexpr int kThreads = 192;
-constexpr int kAtomBytes = 128 * 128;  // one 128-row x 128-byte swizzle atom column (16 KB)
+constexpr int kBM = 128;   // query rows per tile (two tiles per CTA)
+constexpr int kBN = 64;    // keys per block
+constexpr int kThreads = 320;
+constexpr int kQAtom = 128 * 128;  // 128 rows x 128 bytes (16 KB)
+constexpr int kKAtom = 64 * 128;   // 64 rows x 128 bytes (8 KB)
 
 template <int D>
 struct FwdCfg {
-  static constexpr int kAtoms = D / 64;                 // 64-element column atoms per tile row
-  static constexpr int kTileBytes = kAtoms * kAtomBytes;  // a 128 x D bf16 tile
-  static constexpr int kStages = (D == 128) ? 2 : 4;
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kTileBytes;
-  static constexpr int kOffV = kOffK + kStages * kTileBytes;
-  static constexpr int kOffP = kOffV + kStages * kTileBytes;
-  static constexpr int kOffBar = kOffP + 2 * kAtomBytes;  // P is 128 x 128 bf16 = two atoms
-  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 1 + 1 + 1;
+  static constexpr int kAtoms = D / 64;                  // 64-element column atoms per row
+  static constexpr int kQBytes = kAtoms * kQAtom;        // one 128 x D query tile
+  static constexpr int kKVBytes = kAtoms * kKAtom;       // one 64 x D key or value block
+  static constexpr int kStages = (D == 128) ? 3 : 6;  // 224 KB of tiles at D = 128
+  static constexpr int kOffQ = 0;                                  // [2 tiles]
+  static constexpr int kOffK = kOffQ + 2 * kQBytes;                // [stages]
+  static constexpr int kOffV = kOffK + kStages * kKVBytes;         // [stages]
+  static constexpr int kOffP = kOffV + kStages * kKVBytes;         // [tile][buffer] 128 x 64 bf16 = 16 KB
+  static constexpr int kOffBar = kOffP + 4 * kQAtom;
+  static constexpr int kNumBars = 1 + 4 * kStages + 4 + 4 + 4 + 4 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + slack for 1024-byte alignment
-  static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+  // TMEM: S of tile t, buffer u at column 64 * (2t + u); O of tile t at 256 + 128 t.
+  __host__ __device__ static constexpr uint32_t colS(int t, int u) { return 64u * (2 * t + u); }
+  __host__ __device__ static constexpr uint32_t colO(int t) { return 256u + 128u * t; }
 };
 
 struct FwdArgs {
   int B, Hq, Hkv, Sq, Sk;
   int causal;
   float scale_log2;  // softmax scale * log2(e)
-  int n_qtiles;
+  int n_pairs;       // pairs of 128-row query tiles
   uint16_t* o;
   float* lse;
   int* status;
@@ -69,6 +76,14 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
   while (!mbar_try_wait(bar, parity))
     if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
   return true;
+}
+
+// Number of 64-key blocks some row of the 128-row tile starting at `qs` can see.
+__device__ __forceinline__ int tile_blocks(const FwdArgs& a, int qs) {
+  if (qs >= a.Sq) return 0;
+  int kv_end = a.Sk;
+  if (a.causal) kv_end = min(a.Sk, qs + kBM + a.Sk - a.Sq);
+  return kv_end > 0 ? (kv_end + kBN - 1) / kBN : 0;
 }
 
 template <int D>
@@ -88,25 +103,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* k_empty = k_full + C::kStages;
   uint64_t* v_full = k_empty + C::kStages;
   uint64_t* v_empty = v_full + C::kStages;
-  uint64_t* s_full = v_empty + C::kStages;  // [2]
-  uint64_t* s_free = s_full + 2;            // [2]
-  uint64_t* p_full = s_free + 2;
-  uint64_t* o_done = p_full + 1;
-  uint64_t* drain = o_done + 1;
+  uint64_t* s_full = v_empty + C::kStages;  // [tile][buffer]
+  uint64_t* s_free = s_full + 4;            // [tile][buffer]
+  uint64_t* p_full = s_free + 4;            // [tile][P buffer]
+  uint64_t* o_done = p_full + 4;            // [tile][P buffer]: the PV that read that P buffer is done
+  uint64_t* drain = o_done + 4;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // blockIdx.y walks the query tiles from the last (longest under a causal mask) to the first, and
+  // blockIdx.y walks the tile pairs from the last (longest under a causal mask) to the first, and
   // blockIdx.x, which varies fastest in launch order, covers every (batch, head): the longest tiles
   // of all heads start first.
-  const int tile = a.n_qtiles - 1 - static_cast<int>(blockIdx.y);
+  const int pair = a.n_pairs - 1 - static_cast<int>(blockIdx.y);
   const int h = static_cast<int>(blockIdx.x) % a.Hq, b = static_cast<int>(blockIdx.x) / a.Hq;
   const int g = h / (a.Hq / a.Hkv);
-  const int q0 = tile * kBM;
-  int kv_end = a.Sk;  // keys [0, kv_end) can be visible to some row of this tile
-  if (a.causal) kv_end = min(a.Sk, q0 + kBM + a.Sk - a.Sq);
-  const int n_kv = kv_end > 0 ? (kv_end + kBN - 1) / kBN : 0;
+  const int q0 = pair * 2 * kBM;
+  const int n0 = tile_blocks(a, q0), n1 = tile_blocks(a, q0 + kBM);
+  const int nmax = max(n0, n1);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -116,21 +130,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(v_full + s, 1);
       mbar_init(v_empty + s, 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < 4; ++s) {
       mbar_init(s_full + s, 1);
       mbar_init(s_free + s, 4);
     }
-    mbar_init(p_full, 4);
-    mbar_init(o_done, 1);
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(p_full + s, 4);
+      mbar_init(o_done + s, 1);
+    }
     mbar_init(drain, 1);
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
-    tmem_alloc(tmem_holder, C::kTmemCols);
+  if (warp == 9) {
+    tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -140,28 +156,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0 && n_kv > 0) {
-      constexpr uint32_t kBytes = kBM * D * 2;
-      mbar_arrive_expect_tx(q_full, kBytes);
+    if (lane == 0 && nmax > 0) {
+      constexpr uint32_t kQTx = kBM * D * 2;
+      constexpr uint32_t kKVTx = kBN * D * 2;
+      mbar_arrive_expect_tx(q_full, (n0 > 0 ? kQTx : 0u) + (n1 > 0 ? kQTx : 0u));
 #pragma unroll
-      for (int at = 0; at < C::kAtoms; ++at) tma_load_4d(sQ + at * kAtomBytes, &tmQ, q_full, at * 64, h, q0, b);
+      for (int t = 0; t < 2; ++t) {
+        if ((t == 0 ? n0 : n1) == 0) continue;
+#pragma unroll
+        for (int at = 0; at < C::kAtoms; ++at)
+          tma_load_4d(sQ + t * C::kQBytes + at * kQAtom, &tmQ, q_full, at * 64, h, q0 + t * kBM, b);
+      }
       int issued_k = 0, issued_v = 0;
-      for (int j = 0; j < n_kv; ++j) {
+      for (int j = 0; j < nmax; ++j) {
         const int s = j % C::kStages;
         const uint32_t ph = (j / C::kStages) & 1;
         if (!mbar_wait(k_empty + s, ph ^ 1, abort, a.status)) break;
-        mbar_arrive_expect_tx(k_full + s, kBytes);
+        mbar_arrive_expect_tx(k_full + s, kKVTx);
 #pragma unroll
         for (int at = 0; at < C::kAtoms; ++at)
-          tma_load_4d(sK + s * C::kTileBytes + at * kAtomBytes, &tmK, k_full + s, at * 64, g, j * kBN, b);
+          tma_load_4d(sK + s * C::kKVBytes + at * kKAtom, &tmK, k_full + s, at * 64, g, j * kBN, b);
         issued_k = j + 1;
         if (!mbar_wait(v_empty + s, ph ^ 1, abort, a.status)) break;
-        mbar_arrive_expect_tx(v_full + s, kBytes);
+        mbar_arrive_expect_tx(v_full + s, kKVTx);
 #pragma unroll
         for (int at = 0; at < C::kAtoms; ++at)
-          tma_load_4d(sV + s * C::kTileBytes + at * kAtomBytes, &tmV, v_full + s, at * 64, g, j * kBN, b);
+          tma_load_4d(sV + s * C::kKVBytes + at * kKAtom, &tmV, v_full + s, at * 64, g, j * kBN, b);
         issued_v = j + 1;
       }
       // Let every load this thread issued land before the CTA can exit. On the normal path the
@@ -172,45 +194,66 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = max(0, issued_v - C::kStages); j < issued_v; ++j)
         wait_drain(v_full + j % C::kStages, (j / C::kStages) & 1);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_kv > 0) {
+    if (lane == 0 && nmax > 0) {
       constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, 0, 0);
       constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, D, 0, 1);
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+      // base descriptors, built once; each MMA only moves the start address
+      const uint64_t dQ0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dV0 = sdesc_sw128(smem_u32(sV), kKAtom, 1024);
+      const uint64_t dP0 = sdesc_sw128(smem_u32(sP), 16, 1024);
+      const int nt[2] = {n0, n1};
       bool ok = mbar_wait(q_full, 0, abort, a.status);
-      for (int j = 0; ok && j <= n_kv; ++j) {
-        if (j < n_kv) {
+      for (int j = 0; ok && j <= nmax; ++j) {
+        if (j < nmax) {
           const int s = j % C::kStages;
-          const int sb = j & 1;
           if (!mbar_wait(k_full + s, (j / C::kStages) & 1, abort, a.status)) break;
-          if (!mbar_wait(s_free + sb, ((j >> 1) & 1) ^ 1, abort, a.status)) break;
-          tc_fence_after();
-          const uint32_t dS = tmem + (sb ? C::kColS1 : C::kColS0);
+          const uint64_t dK = sdesc_advance(dK0, s * C::kKVBytes);
+          for (int t = 0; t < 2; ++t) {
+            if (j >= nt[t]) continue;
+            const int u = j & 1;
+            if (!mbar_wait(s_free + 2 * t + u, ((j >> 1) & 1) ^ 1, abort, a.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t dQ = sdesc_advance(dQ0, t * C::kQBytes);
+            const uint32_t dS = tmem + C::colS(t, u);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kAtomBytes + (kk & 3) * 32;
-            umma_ss(dS, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + s * C::kTileBytes + off, 16, 1024),
-                    kIdescS, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              umma_ss(dS, sdesc_advance(dQ, (kk >> 2) * kQAtom + (kk & 3) * 32),
+                      sdesc_advance(dK, (kk >> 2) * kKAtom + (kk & 3) * 32), kIdescS, kk > 0);
+            }
+            umma_commit(s_full + 2 * t + u);
           }
-          umma_commit(s_full + sb);
+          if (!ok) break;
           umma_commit(k_empty + s);
         }
         if (j >= 1) {
           const int jj = j - 1;
           const int s = jj % C::kStages;
-          if (!mbar_wait(p_full, jj & 1, abort, a.status)) break;
           if (!mbar_wait(v_full + s, (jj / C::kStages) & 1, abort, a.status)) break;
-          tc_fence_after();
+          const uint64_t dV = sdesc_advance(dV0, s * C::kKVBytes);
+          for (int t = 0; t < 2; ++t) {
+            if (jj >= nt[t]) continue;
+            const int pb = jj & 1;  // P buffer of block jj
+            if (!mbar_wait(p_full + 2 * t + pb, (jj >> 1) & 1, abort, a.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t dP = sdesc_advance(dP0, (2 * t + pb) * kQAtom);
+            const uint32_t dO = tmem + C::colO(t);
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk) {
-            const uint32_t offp = (kk >> 2) * kAtomBytes + (kk & 3) * 32;
-            const uint32_t offv = kk * 16 * 128;  // 16 key rows of 128 bytes
-            umma_ss(tmem + C::kColO, sdesc_sw128(aP + offp, 16, 1024),
-                    sdesc_sw128(aV + s * C::kTileBytes + offv, kAtomBytes, 1024), kIdescO, (jj > 0 || kk > 0));
+            for (int kk = 0; kk < kBN / 16; ++kk) {
+              umma_ss(dO, sdesc_advance(dP, kk * 32), sdesc_advance(dV, kk * 16 * 128), kIdescO, (jj > 0 || kk > 0));
+            }
+            umma_commit(o_done + 2 * t + pb);
           }
+          if (!ok) break;
           umma_commit(v_empty + s);
-          umma_commit(o_done);
         }
       }
       // all MMAs issued by this thread complete before the CTA releases TMEM
@@ -218,12 +261,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_drain(drain, 0);
     }
   } else {
-    // ------------------------------------------------------------------ softmax warpgroup
-    const int row = threadIdx.x;  // 0..127 == TMEM lane
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
-    const int qrow = q0 + row;
+    // ------------------------------------------------------------------ softmax warpgroups
+    const int t = warp >> 2;               // query tile of this warpgroup
+    const int row = threadIdx.x & 127;     // TMEM lane == row in the tile
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int n_kv = t == 0 ? n0 : n1;
+    const int qrow = q0 + t * kBM + row;
     int row_limit = a.Sk - 1;  // largest visible key index for this row
     if (a.causal) row_limit = min(row_limit, qrow + a.Sk - a.Sq);
+    uint8_t* myP = sP + 2 * t * kQAtom;  // this tile's two P buffers
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     // every lane waits; the outcome is made warp-uniform before any warp-collective tcgen05 op
@@ -232,80 +278,90 @@ __global__ void __launch_bounds__(kThreads, 1)
       return __all_sync(0xffffffffu, r);
     };
     for (int j = 0; j < n_kv; ++j) {
-      const int sb = j & 1;
-      if (!wait_warp(s_full + sb, (j >> 1) & 1)) {
+      const int u = j & 1;
+      if (!wait_warp(s_full + 2 * t + u, (j >> 1) & 1)) {
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t sr[kBN];
 #pragma unroll
-      for (int c = 0; c < kBN / 16; ++c) tmem_ld16(tmem + lane_addr + (sb ? C::kColS1 : C::kColS0) + c * 16, sr + c * 16);
+      for (int c = 0; c < kBN / 16; ++c) tmem_ld16(tmem + lane_addr + C::colS(t, u) + c * 16, sr + c * 16);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(s_free + sb);
+      if (lane == 0) mbar_arrive(s_free + 2 * t + u);
 
       const int kbase = j * kBN;
       const bool need_mask = kbase + kBN - 1 > row_limit;
-      float mx = -INFINITY;
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four independent max chains
 #pragma unroll
       for (int c = 0; c < kBN; ++c) {
         float x = __uint_as_float(sr[c]) * a.scale_log2;
         if (need_mask && kbase + c > row_limit) x = -INFINITY;
         sr[c] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+        mx4[c & 3] = fmaxf(mx4[c & 3], x);
       }
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       // lazy rescale: move the reference max only when the block max exceeds it by more than 8
       float alpha = 1.f;
       if (mx > m + 8.f || (m == -INFINITY && mx != -INFINITY)) {
-        alpha = (m == -INFINITY) ? 0.f : exp2f(m - mx);
+        alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - mx);
         m = mx;
       }
       const float m_use = (m == -INFINITY) ? 0.f : m;
-      float rs = 0.f;
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent sum chains
       uint32_t pk[kBN / 2];
 #pragma unroll
       for (int c = 0; c < kBN; c += 2) {
-        const float p0 = exp2f(__uint_as_float(sr[c]) - m_use);
-        const float p1 = exp2f(__uint_as_float(sr[c + 1]) - m_use);
-        rs += p0 + p1;
+        const float p0 = fast_exp2(__uint_as_float(sr[c]) - m_use);
+        const float p1 = fast_exp2(__uint_as_float(sr[c + 1]) - m_use);
+        rs4[(c >> 1) & 3] += p0 + p1;
         pk[c / 2] = pack_bf16(p0, p1);
       }
-      l = l * alpha + rs;
+      l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
 
-      // PV_{j-1} must be complete before O is rescaled and before P's buffer is overwritten.
-      if (j >= 1) {
-        if (!wait_warp(o_done, (j - 1) & 1)) {
+      // P buffer j & 1 was last read by the PV of block j - 2: wait for it before overwriting.
+      const int pb = j & 1;
+      if (j >= 2) {
+        if (!wait_warp(o_done + 2 * t + pb, ((j - 2) >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+      }
+      // O may be rescaled only once the PV of block j - 1 has landed (rare with lazy rescaling).
+      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (!wait_warp(o_done + 2 * t + (pb ^ 1), ((j - 1) >> 1) & 1)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        {
 #pragma unroll 1
           for (int c0 = 0; c0 < D; c0 += 16) {
             uint32_t orr[16];
-            tmem_ld16(tmem + lane_addr + C::kColO + c0, orr);
+            tmem_ld16(tmem + lane_addr + C::colO(t) + c0, orr);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 16; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-            tmem_st16(tmem + lane_addr + C::kColO + c0, orr);
+            tmem_st16(tmem + lane_addr + C::colO(t) + c0, orr);
           }
           tmem_wait_st();
         }
       }
-      // P row -> shared memory, 128-byte swizzled K-major (two 64-key atoms)
+      // P row -> shared memory, 128-byte swizzled K-major (one 64-key atom)
 #pragma unroll
       for (int ch = 0; ch < kBN / 8; ++ch) {
-        uint4 w = make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-        *reinterpret_cast<uint4*>(sP + (ch >> 3) * kAtomBytes + sw128_offset(row, ch & 7)) = w;
+        *reinterpret_cast<uint4*>(myP + pb * kQAtom + sw128_offset(row, ch)) =
+            make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(p_full + 2 * t + pb);
     }
-    if (ok && n_kv > 0) ok = wait_warp(o_done, (n_kv - 1) & 1);
+    // the last PV of this tile (it was issued after every earlier one)
+    if (ok && n_kv > 0) ok = wait_warp(o_done + 2 * t + ((n_kv - 1) & 1), ((n_kv - 1) >> 1) & 1);
     tc_fence_after();
     // epilogue: O / l -> bf16, lse = (m + log2 l) ln 2
     const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -315,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c0 = 0; c0 < D; c0 += 16) {
       uint32_t orr[16];
       if (ok && n_kv > 0) {
-        tmem_ld16(tmem + lane_addr + C::kColO + c0, orr);
+        tmem_ld16(tmem + lane_addr + C::colO(t) + c0, orr);
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -340,9 +396,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -354,8 +410,8 @@ cudaError_t launch_fwd_sm100_d(const Problem& p, const void* q, const void* k, c
                                cudaStream_t st) {
   using C = FwdCfg<D>;
   CUtensorMap mq, mk, mv;
-  if (!make_map_bf16_sw128(&mq, q, p.B, p.Sq, p.Hq, D, kBM) || !make_map_bf16_sw128(&mk, k, p.B, p.Sk, p.Hkv, D, kBN) ||
-      !make_map_bf16_sw128(&mv, v, p.B, p.Sk, p.Hkv, D, kBN))
+  if (!make_map_bf16_sw128(&mq, q, p.B, p.Sq, p.Hq, D, kBM) ||
+      !make_map_bf16_sw128(&mk, k, p.B, p.Sk, p.Hkv, D, kBN) || !make_map_bf16_sw128(&mv, v, p.B, p.Sk, p.Hkv, D, kBN))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
@@ -367,11 +423,11 @@ cudaError_t launch_fwd_sm100_d(const Problem& p, const void* q, const void* k, c
   a.Sk = p.Sk;
   a.causal = p.causal;
   a.scale_log2 = p.scale * kLog2e;
-  a.n_qtiles = (p.Sq + kBM - 1) / kBM;
+  a.n_pairs = (p.Sq + 2 * kBM - 1) / (2 * kBM);
   a.o = static_cast<uint16_t*>(o);
   a.lse = lse;
   a.status = device_status_ptr();
-  dim3 grid(p.Hq * p.B, a.n_qtiles);
+  dim3 grid(p.Hq * p.B, a.n_pairs);
   {
     LaunchScope ls("fwd_sm100", st);
     fwd_sm100_kernel<D><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);

@@ -27,7 +27,7 @@
 // epilogue), warps 4-7 dQ drain (one TMEM lane per thread: tcgen05.ld -> shared -> per-warp TMA
 // reduce-add of 32 columns),
 // warp 8 TMA producer (K, V once; Q and dO tiles through a ring), warp 9 TMEM allocator and MMA
-// issuer. The MMA issuer puts the next tile's S^T/dP^T ahead of the current tile's gradient MMAs
+// issuer (one elected lane). The MMA issuer puts the next tile's S^T/dP^T ahead of the current tile's gradient MMAs
 // so that the tensor cores work while the score warps compute P and dS. Every wait is bounded.
 #include <math.h>
 
@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_it > 0) {
+    if (n_it > 0) {  // the whole warp runs the loop; one elected lane issues each MMA
       constexpr uint32_t kIdS = idesc_bf16_f32(kBN, kBM, 0, 0);  // S^T, dP^T
       constexpr uint32_t kIdG = idesc_bf16_f32(kBN, D, 0, 1);    // dV, dK
       constexpr uint32_t kIdQ = idesc_bf16_f32(128, kBM, 1, 1);  // dQ^T (M = 128 also for D = 64)
@@ -209,28 +209,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t mDO = sdesc_sw128(smem_u32(sDO), kQAtom, 1024);
       const uint64_t mK = sdesc_sw128(smem_u32(sK), kKAtom, 1024);
       const uint64_t mDS = sdesc_sw128(smem_u32(sDS), kQAtom, 1024);
-      bool ok = mbar_wait(kv_full, 0, abort, a.status);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(kv_full, 0, abort, a.status));
       for (int j = 0; ok && j <= n_it; ++j) {
         if (j < n_it) {
           const int s = j % C::kStages;
-          if (!mbar_wait(q_full + s, (j / C::kStages) & 1, abort, a.status)) break;
-          if (!mbar_wait(st_free, (j & 1) ^ 1, abort, a.status)) break;
+          if (!__all_sync(0xffffffffu, mbar_wait(q_full + s, (j / C::kStages) & 1, abort, a.status))) break;
+          if (!__all_sync(0xffffffffu, mbar_wait(st_free, (j & 1) ^ 1, abort, a.status))) break;
           tc_fence_after();
           const uint64_t q = sdesc_advance(kQ, s * C::kQBytes), dO = sdesc_advance(kDO, s * C::kQBytes);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t ok_ = (kk >> 2) * kKAtom + (kk & 3) * 32;
             const uint32_t oq = (kk >> 2) * kQAtom + (kk & 3) * 32;
-            umma_ss(tmem + C::kColS, sdesc_advance(kK, ok_), sdesc_advance(q, oq), kIdS, kk > 0);
-            umma_ss(tmem + C::kColDP, sdesc_advance(kV, ok_), sdesc_advance(dO, oq), kIdS, kk > 0);
+            umma_ss_warp(tmem + C::kColS, sdesc_advance(kK, ok_), sdesc_advance(q, oq), kIdS, kk > 0);
+            umma_ss_warp(tmem + C::kColDP, sdesc_advance(kV, ok_), sdesc_advance(dO, oq), kIdS, kk > 0);
           }
-          umma_commit(s_full);
+          umma_commit_warp(s_full);
         }
         if (j >= 1) {
           const int jj = j - 1;
           const int s = jj % C::kStages;
-          if (!mbar_wait(p_full, jj & 1, abort, a.status)) break;
-          if (!mbar_wait(dq_free, (jj & 1) ^ 1, abort, a.status)) break;
+          if (!__all_sync(0xffffffffu, mbar_wait(p_full, jj & 1, abort, a.status))) break;
+          if (!__all_sync(0xffffffffu, mbar_wait(dq_free, (jj & 1) ^ 1, abort, a.status))) break;
           tc_fence_after();
           const uint64_t q = sdesc_advance(mQ, s * C::kQBytes), dO = sdesc_advance(mDO, s * C::kQBytes);
           // dV += P^T dO, dK += dS^T Q: K = 64 query rows in 4 steps of 16
@@ -239,23 +239,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t oa = kk * 32;          // 16 rows = 32 bytes along the swizzled K-major row
             const uint32_t ob = kk * 16 * 128;    // 16 rows of 128 bytes in the MN-major operand
             const uint32_t acc = (jj > 0 || kk > 0);
-            umma_ss(tmem + C::kColDV, sdesc_advance(kP, oa), sdesc_advance(dO, ob), kIdG, acc);
-            umma_ss(tmem + C::kColDK, sdesc_advance(kDS, oa), sdesc_advance(q, ob), kIdG, acc);
+            umma_ss_warp(tmem + C::kColDV, sdesc_advance(kP, oa), sdesc_advance(dO, ob), kIdG, acc);
+            umma_ss_warp(tmem + C::kColDK, sdesc_advance(kDS, oa), sdesc_advance(q, ob), kIdG, acc);
           }
           // dQ^T = K^T dS^T: K = 128 keys in 8 steps of 16
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
             const uint32_t o = kk * 16 * 128;
-            umma_ss(tmem + C::kColDQ, sdesc_advance(mK, o), sdesc_advance(mDS, o), kIdQ, kk > 0);
+            umma_ss_warp(tmem + C::kColDQ, sdesc_advance(mK, o), sdesc_advance(mDS, o), kIdQ, kk > 0);
           }
-          umma_commit(q_empty + s);
-          umma_commit(pds_free);
-          umma_commit(dq_full);
+          umma_commit_warp(q_empty + s);
+          umma_commit_warp(pds_free);
+          umma_commit_warp(dq_full);
         }
       }
-      umma_commit(all_done);
-      umma_commit(drain);
+      umma_commit_warp(all_done);
+      umma_commit_warp(drain);
       wait_drain(drain, 0);
+      __syncwarp();
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------------ score warps (row = key)

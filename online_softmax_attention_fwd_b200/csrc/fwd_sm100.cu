@@ -17,7 +17,7 @@
 //                    grows by more than 2^8, epilogue O / l and lse. With two P buffers per tile the
 //                    softmax waits for a PV only when it must rescale O.
 //   warp 8           TMA producer: both Q tiles once, then K and V blocks through a ring.
-//   warp 9           TMEM allocator and MMA issuer (one thread): S of block j for both tiles
+//   warp 9           TMEM allocator and MMA issuer (one elected lane): S of block j for both tiles
 //                    (double-buffered in TMEM), then P V of block j - 1 for both tiles, so that the
 //                    tensor cores work on one tile while the other tile's softmax runs.
 // Lazy rescaling: a row keeps its old max m while the block max stays within m + 8 (base 2); P then
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0 && nmax > 0) {
+    if (nmax > 0) {  // the whole warp runs the loop; one elected lane issues each MMA
       constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, 0, 0);
       constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, D, 0, 1);
       // base descriptors, built once; each MMA only moves the start address
@@ -205,16 +205,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dV0 = sdesc_sw128(smem_u32(sV), kKAtom, 1024);
       const uint64_t dP0 = sdesc_sw128(smem_u32(sP), 16, 1024);
       const int nt[2] = {n0, n1};
-      bool ok = mbar_wait(q_full, 0, abort, a.status);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort, a.status));
       for (int j = 0; ok && j <= nmax; ++j) {
         if (j < nmax) {
           const int s = j % C::kStages;
-          if (!mbar_wait(k_full + s, (j / C::kStages) & 1, abort, a.status)) break;
+          if (!__all_sync(0xffffffffu, mbar_wait(k_full + s, (j / C::kStages) & 1, abort, a.status))) break;
           const uint64_t dK = sdesc_advance(dK0, s * C::kKVBytes);
           for (int t = 0; t < 2; ++t) {
             if (j >= nt[t]) continue;
             const int u = j & 1;
-            if (!mbar_wait(s_free + 2 * t + u, ((j >> 1) & 1) ^ 1, abort, a.status)) {
+            if (!__all_sync(0xffffffffu, mbar_wait(s_free + 2 * t + u, ((j >> 1) & 1) ^ 1, abort, a.status))) {
               ok = false;
               break;
             }
@@ -223,23 +223,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t dS = tmem + C::colS(t, u);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-              umma_ss(dS, sdesc_advance(dQ, (kk >> 2) * kQAtom + (kk & 3) * 32),
+              umma_ss_warp(dS, sdesc_advance(dQ, (kk >> 2) * kQAtom + (kk & 3) * 32),
                       sdesc_advance(dK, (kk >> 2) * kKAtom + (kk & 3) * 32), kIdescS, kk > 0);
             }
-            umma_commit(s_full + 2 * t + u);
+            umma_commit_warp(s_full + 2 * t + u);
           }
           if (!ok) break;
-          umma_commit(k_empty + s);
+          umma_commit_warp(k_empty + s);
         }
         if (j >= 1) {
           const int jj = j - 1;
           const int s = jj % C::kStages;
-          if (!mbar_wait(v_full + s, (jj / C::kStages) & 1, abort, a.status)) break;
+          if (!__all_sync(0xffffffffu, mbar_wait(v_full + s, (jj / C::kStages) & 1, abort, a.status))) break;
           const uint64_t dV = sdesc_advance(dV0, s * C::kKVBytes);
           for (int t = 0; t < 2; ++t) {
             if (jj >= nt[t]) continue;
             const int pb = jj & 1;  // P buffer of block jj
-            if (!mbar_wait(p_full + 2 * t + pb, (jj >> 1) & 1, abort, a.status)) {
+            if (!__all_sync(0xffffffffu, mbar_wait(p_full + 2 * t + pb, (jj >> 1) & 1, abort, a.status))) {
               ok = false;
               break;
             }
@@ -248,17 +248,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t dO = tmem + C::colO(t);
 #pragma unroll
             for (int kk = 0; kk < kBN / 16; ++kk) {
-              umma_ss(dO, sdesc_advance(dP, kk * 32), sdesc_advance(dV, kk * 16 * 128), kIdescO, (jj > 0 || kk > 0));
+              umma_ss_warp(dO, sdesc_advance(dP, kk * 32), sdesc_advance(dV, kk * 16 * 128), kIdescO, (jj > 0 || kk > 0));
             }
-            umma_commit(o_done + 2 * t + pb);
+            umma_commit_warp(o_done + 2 * t + pb);
           }
           if (!ok) break;
-          umma_commit(v_empty + s);
+          umma_commit_warp(v_empty + s);
         }
       }
       // all MMAs issued by this thread complete before the CTA releases TMEM
-      umma_commit(drain);
+      umma_commit_warp(drain);
       wait_drain(drain, 0);
+      __syncwarp();
     }
   } else {
     // ------------------------------------------------------------------ softmax warpgroups

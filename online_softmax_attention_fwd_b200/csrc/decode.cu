@@ -10,14 +10,23 @@
 // kernel uses between its four warps, so the result does not depend on how the keys were cut.
 //
 // The path is HBM-bound (each K/V byte is read once, about 4 flop per byte), so the split kernel is
-// CUDA-core code built for bytes in flight: a CTA covers one (chunk, kv head, stream) and all the
-// query heads of that kv head's group, so each K/V row is fetched once for GT query heads. Each
-// lane scores one key (16-byte vector loads of its K row) and owns D/32 value dimensions (coalesced
-// V rows); a block's V loads are issued before its softmax arithmetic so that they overlap it.
+// CUDA-core code built to keep many bytes in flight without spending registers on them. A CTA
+// covers one (chunk, kv head, stream) and all the query heads of that kv head's group, so each K/V
+// row is fetched once for GT query heads. One producer warp streams 32-key K and V blocks of the
+// chunk with TMA tile loads (128-byte swizzle) into a 4-stage shared-memory ring; compute warp w
+// takes blocks w, w+4, ... and keeps its own online-softmax triples for the GT heads: each lane
+// scores one key for all GT heads (its K row read once from shared memory) and owns D/32 value
+// dimensions of every head (each V row read once per lane). The four warps' triples are merged
+// with the monoid at the end.
+// The host does not know the cache's row count T (it lives on the device as kv_offsets[N]), so the
+// tensor maps carry a nominal row extent and the kernel issues a 32-row box only when the whole box
+// lies below T; the cache's last partial block is fetched in 16-byte pieces with bulk copies. No
+// copy ever touches memory past the caller's K and V buffers.
 #include <math.h>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tma_host.h"
 
 namespace attn {
 
@@ -47,38 +56,51 @@ __device__ __forceinline__ int stream_splits(const int* num_splits, int n, int L
   return decode_split_rule(L, max_splits);
 }
 
-template <int DPL>
-struct VPiece;
-template <>
-struct VPiece<4> {
-  uint32_t w[2];
-  __device__ __forceinline__ void load(const uint16_t* p) {
-    const uint2 x = __ldg(reinterpret_cast<const uint2*>(p));
-    w[0] = x.x;
-    w[1] = x.y;
-  }
-  __device__ __forceinline__ void zero() { w[0] = w[1] = 0u; }
-  __device__ __forceinline__ float get(int i) const { return (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]); }
-};
-template <>
-struct VPiece<2> {
-  uint32_t w[1];
-  __device__ __forceinline__ void load(const uint16_t* p) { w[0] = __ldg(reinterpret_cast<const unsigned*>(p)); }
-  __device__ __forceinline__ void zero() { w[0] = 0u; }
-  __device__ __forceinline__ float get(int i) const { return (i & 1) ? bf16_hi(w[0]) : bf16_lo(w[0]); }
+constexpr int kDecBlk = 32;              // keys per block (one per lane)
+constexpr int kDecStages = 4;
+constexpr int kDecThreads = 160;          // four compute warps + one producer warp
+constexpr int kDecMapRows = 0x7fffffff;   // nominal row extent of the K/V tensor maps
+
+template <int D>
+struct DecCfg {
+  static constexpr int kAtoms = D / 64;
+  static constexpr int kAtomBytes = kDecBlk * 128;       // 32 rows x 128 bytes
+  static constexpr int kBlkBytes = kAtoms * kAtomBytes;  // 32 key rows x D bf16
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kDecStages * kBlkBytes;
+  static constexpr int kOffBar = 2 * kDecStages * kBlkBytes;
+  static constexpr int kSmemBytes = kOffBar + 2 * kDecStages * 8 + 16 + 1024;
 };
 
+__device__ __forceinline__ bool dec_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  return true;
+}
+
+// Byte offset of element d of row r in a 128-byte-swizzled block of 64-element column atoms.
+template <int D>
+__device__ __forceinline__ uint32_t dec_sw(int r, int d) {
+  return (d >> 6) * DecCfg<D>::kAtomBytes + sw128_offset(r, (d & 63) >> 3) + (d & 7) * 2;
+}
+
 template <int D, int GT>
-__global__ void __launch_bounds__(128) decode_split_kernel(const uint16_t* __restrict__ q,
-                                                           const uint16_t* __restrict__ k,
-                                                           const uint16_t* __restrict__ v,
-                                                           const int* __restrict__ offsets,
-                                                           const int* __restrict__ num_splits, int max_splits,
-                                                           int Hq, int Hkv, float scale_log2,
-                                                           float* __restrict__ part_o,
-                                                           float* __restrict__ part_ml) {
-  constexpr int KV16 = D / 8;  // 16-byte pieces per K row
+__global__ void __launch_bounds__(kDecThreads, 3)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                        const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
+                        const uint16_t* __restrict__ v, const int* __restrict__ offsets, int N,
+                        const int* __restrict__ num_splits, int max_splits, int Hq, int Hkv, float scale_log2,
+                        float* __restrict__ part_o, float* __restrict__ part_ml, int* status) {
+  using C = DecCfg<D>;
   constexpr int DPL = D / 32;  // value dimensions per lane
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem + C::kOffK;
+  uint8_t* sV = smem + C::kOffV;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* empty = full + kDecStages;
+  volatile int* abort = reinterpret_cast<volatile int*>(empty + kDecStages);
   __shared__ __align__(16) float qs[GT][D];
   __shared__ float red_m[4][GT];
   __shared__ float red_l[4][GT];
@@ -90,20 +112,72 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const uint16_t* __res
   const int h0 = g * G + (blockIdx.y % npass) * GT;
   const int start = offsets[n];
   const int L = offsets[n + 1] - start;
-  const int C = stream_splits(num_splits, n, L, max_splits);
-  if (c >= C) return;  // uniform over the CTA; the combine reads only the first C slots
-  const int chunk = (L + C - 1) / C;
+  const int C_n = stream_splits(num_splits, n, L, max_splits);
+  if (c >= C_n) return;  // uniform over the CTA; the combine reads only the first C_n slots
+  const int chunk = (L + C_n - 1) / C_n;
   const int k0 = min(L, c * chunk);
   const int k1 = min(L, k0 + chunk);
+  const int nblk = (k1 - k0 + kDecBlk - 1) / kDecBlk;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int e = tid; e < GT * D; e += 128) {
+  if (tid == 0) {
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);  // each block is consumed by exactly one compute warp
+    }
+    *abort = 0;
+    fence_mbar_init();
+  }
+  for (int e = tid; e < GT * D; e += kDecThreads) {
     const int t = e / D, d = e - t * D;
     qs[t][d] = __uint_as_float(static_cast<uint32_t>(q[(static_cast<long long>(n) * Hq + h0 + t) * D + d]) << 16) *
                scale_log2;
   }
   __syncthreads();
 
+  if (warp == 4) {
+    // ---------------------------------------------------------------- producer
+    const int T = min(offsets[N], kDecMapRows);  // no box may reach past the cache
+    const long long rs = static_cast<long long>(Hkv) * D;
+    int issued = 0;
+    for (int bk = 0; bk < nblk; ++bk) {
+      const int s = bk % kDecStages;
+      const int row0 = start + k0 + bk * kDecBlk;
+      const bool tile = row0 + kDecBlk <= T;
+      const int nrows = tile ? kDecBlk : min(kDecBlk, k1 - (k0 + bk * kDecBlk));
+      bool ok = true;
+      if (lane == 0) {
+        ok = mbar_wait(empty + s, ((bk / kDecStages) & 1) ^ 1, abort, status);
+        if (ok) {
+          mbar_arrive_expect_tx(full + s, 2u * nrows * D * 2);
+          if (tile) {
+#pragma unroll
+            for (int at = 0; at < C::kAtoms; ++at) {
+              tma_load_3d(sK + s * C::kBlkBytes + at * C::kAtomBytes, &tmK, full + s, at * 64, g, row0);
+              tma_load_3d(sV + s * C::kBlkBytes + at * C::kAtomBytes, &tmV, full + s, at * 64, g, row0);
+            }
+          }
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+      if (!tile) {
+        // the cache's last rows: 16-byte pieces into the same swizzled places a tile load uses
+        for (int idx = lane; idx < nrows * (D / 8); idx += 32) {
+          const int r = idx / (D / 8), d = (idx % (D / 8)) * 8;
+          bulk_load(sK + s * C::kBlkBytes + dec_sw<D>(r, d), k + (row0 + r) * rs + g * D + d, 16, full + s);
+          bulk_load(sV + s * C::kBlkBytes + dec_sw<D>(r, d), v + (row0 + r) * rs + g * D + d, 16, full + s);
+        }
+      }
+      issued = bk + 1;
+    }
+    // let this CTA's copies land before it can exit (at once on the normal path)
+    if (lane == 0)
+      for (int bk = max(0, issued - kDecStages); bk < issued; ++bk)
+        dec_wait_drain(full + bk % kDecStages, (bk / kDecStages) & 1);
+    return;
+  }
+
+  // ------------------------------------------------------------------ compute warps
   float m[GT], ls[GT], acc[GT][DPL];
 #pragma unroll
   for (int t = 0; t < GT; ++t) {
@@ -112,81 +186,78 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const uint16_t* __res
 #pragma unroll
     for (int e = 0; e < DPL; ++e) acc[t][e] = 0.f;
   }
-  const long long rs = static_cast<long long>(Hkv) * D;
-  const uint16_t* kb = k + (static_cast<long long>(start) * Hkv + g) * D;
-  const uint16_t* vb = v + (static_cast<long long>(start) * Hkv + g) * D + lane * DPL;
-
-  for (int base = k0 + 32 * warp; base < k1; base += 128) {
-    const int j = base + lane;
-    const bool valid = j < k1;
-    const int nk = min(32, k1 - base);
-    uint4 kr[KV16];
-    if (valid) {
-      const uint4* src = reinterpret_cast<const uint4*>(kb + j * rs);
+  const int vd = lane * DPL;  // this lane's value dimensions: vd .. vd + DPL - 1
+  for (int bk = warp; bk < nblk; bk += 4) {
+    const int s = bk % kDecStages;
+    const bool ok = mbar_wait(full + s, (bk / kDecStages) & 1, abort, status);
+    if (!__all_sync(0xffffffffu, ok)) break;
+    const uint8_t* kb = sK + s * C::kBlkBytes;
+    const uint8_t* vb = sV + s * C::kBlkBytes;
+    const int nk = min(kDecBlk, k1 - (k0 + bk * kDecBlk));
+    const bool valid = lane < nk;
+    // scores of this lane's key for the GT heads (base-2 units: q carries scale * log2 e)
+    float sc[GT];
 #pragma unroll
-      for (int x = 0; x < KV16; ++x) kr[x] = __ldg(src + x);
-    } else {
+    for (int t = 0; t < GT; ++t) sc[t] = 0.f;
 #pragma unroll
-      for (int x = 0; x < KV16; ++x) kr[x] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    // scores of this lane's key for the GT query heads (base-2 units: q carries scale * log2 e)
-    float s[GT];
-#pragma unroll
-    for (int t = 0; t < GT; ++t) s[t] = 0.f;
-#pragma unroll
-    for (int x = 0; x < KV16; ++x) {
-      const uint32_t w[4] = {kr[x].x, kr[x].y, kr[x].z, kr[x].w};
+    for (int cc = 0; cc < D / 8; ++cc) {
+      const uint4 w = *reinterpret_cast<const uint4*>(kb + dec_sw<D>(lane, cc * 8));
+      const float k_[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                           bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
 #pragma unroll
       for (int t = 0; t < GT; ++t) {
-        const float4 qa = *reinterpret_cast<const float4*>(&qs[t][8 * x]);
-        const float4 qb = *reinterpret_cast<const float4*>(&qs[t][8 * x + 4]);
-        float a = s[t];
-        a = fmaf(qa.x, bf16_lo(w[0]), a);
-        a = fmaf(qa.y, bf16_hi(w[0]), a);
-        a = fmaf(qa.z, bf16_lo(w[1]), a);
-        a = fmaf(qa.w, bf16_hi(w[1]), a);
-        a = fmaf(qb.x, bf16_lo(w[2]), a);
-        a = fmaf(qb.y, bf16_hi(w[2]), a);
-        a = fmaf(qb.z, bf16_lo(w[3]), a);
-        a = fmaf(qb.w, bf16_hi(w[3]), a);
-        s[t] = a;
+        const float4 qa = *reinterpret_cast<const float4*>(&qs[t][8 * cc]);
+        const float4 qb = *reinterpret_cast<const float4*>(&qs[t][8 * cc + 4]);
+        float x = sc[t];
+        x = fmaf(qa.x, k_[0], x);
+        x = fmaf(qa.y, k_[1], x);
+        x = fmaf(qa.z, k_[2], x);
+        x = fmaf(qa.w, k_[3], x);
+        x = fmaf(qb.x, k_[4], x);
+        x = fmaf(qb.y, k_[5], x);
+        x = fmaf(qb.z, k_[6], x);
+        x = fmaf(qb.w, k_[7], x);
+        sc[t] = x;
       }
-    }
-    // V loads go out before the softmax arithmetic so that they overlap it
-    VPiece<DPL> vr[32];
-#pragma unroll
-    for (int jj = 0; jj < 32; ++jj) {
-      if (jj < nk)
-        vr[jj].load(vb + (base + jj) * rs);
-      else
-        vr[jj].zero();
     }
     float p[GT];
 #pragma unroll
     for (int t = 0; t < GT; ++t) {
-      const float st = valid ? s[t] : -INFINITY;
+      const float st = valid ? sc[t] : -INFINITY;
       const float mn = fmaxf(m[t], warp_max(st));  // finite: lane 0's key is valid
-      const float alpha = exp2f(m[t] - mn);         // 2^(-inf) = 0 on the first block
-      p[t] = valid ? exp2f(st - mn) : 0.f;
+      const float alpha = fast_exp2(m[t] - mn);     // 2^(-inf) = 0 on the first block
+      p[t] = valid ? fast_exp2(st - mn) : 0.f;
       ls[t] = ls[t] * alpha + p[t];
 #pragma unroll
       for (int e = 0; e < DPL; ++e) acc[t][e] *= alpha;
       m[t] = mn;
     }
+    for (int j = 0; j < nk; ++j) {
+      const uint8_t* vr = vb + dec_sw<D>(j, vd);
+      float vv[DPL];
+      if constexpr (DPL == 4) {
+        const uint2 w = *reinterpret_cast<const uint2*>(vr);
+        vv[0] = bf16_lo(w.x);
+        vv[1] = bf16_hi(w.x);
+        vv[2] = bf16_lo(w.y);
+        vv[3] = bf16_hi(w.y);
+      } else {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(vr);
+        vv[0] = bf16_lo(w);
+        vv[1] = bf16_hi(w);
+      }
 #pragma unroll
-    for (int jj = 0; jj < 32; ++jj) {
-      if (jj < nk) {
+      for (int t = 0; t < GT; ++t) {
+        const float pj = __shfl_sync(0xffffffffu, p[t], j);
 #pragma unroll
-        for (int t = 0; t < GT; ++t) {
-          const float pj = __shfl_sync(0xffffffffu, p[t], jj);
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) acc[t][e] = fmaf(pj, vr[jj].get(e), acc[t][e]);
-        }
+        for (int e = 0; e < DPL; ++e) acc[t][e] = fmaf(pj, vv[e], acc[t][e]);
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty + s);
   }
 
-  // merge the four warps' triples (a warp that saw no key holds the identity)
+  // merge the four warps' triples (a warp that saw no block holds the identity)
 #pragma unroll
   for (int t = 0; t < GT; ++t) {
     const float lw = warp_sum(ls[t]);
@@ -195,9 +266,9 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const uint16_t* __res
       red_l[warp][t] = lw;
     }
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) red_o[warp][t][lane * DPL + e] = acc[t][e];
+    for (int e = 0; e < DPL; ++e) red_o[warp][t][vd + e] = acc[t][e];
   }
-  __syncthreads();
+  named_barrier(1, 128);  // the four compute warps only
   for (int e = tid; e < GT * D; e += 128) {
     const int t = e / D, d = e - t * D;
     float M = -INFINITY;
@@ -208,7 +279,7 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const uint16_t* __res
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
         const float mw = red_m[w][t];
-        const float wt = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+        const float wt = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
         Lsum = fmaf(wt, red_l[w][t], Lsum);
         O = fmaf(wt, red_o[w][t][d], O);
       }
@@ -291,15 +362,20 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
 
 template <int D, int GT>
 cudaError_t launch_split(const DecodeProblem& p, const void* q, const void* k, const void* v,
-                         const int* offsets, const int* num_splits, float* part_o, float* part_ml,
-                         cudaStream_t st) {
+                         const CUtensorMap& mk, const CUtensorMap& mv, const int* offsets, const int* num_splits,
+                         float* part_o, float* part_ml, cudaStream_t st) {
+  using C = DecCfg<D>;
   const int npass = (p.Hq / p.Hkv) / GT;
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, GT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::kSmemBytes);
+  if (e != cudaSuccess) return e;
   dim3 grid(p.max_splits, p.Hkv * npass, p.N);
   {
     LaunchScope ls("decode_split", st);
-    decode_split_kernel<D, GT><<<grid, 128, 0, st>>>(
-        static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v),
-        offsets, num_splits, p.max_splits, p.Hq, p.Hkv, p.scale * kLog2e, part_o, part_ml);
+    decode_split_kernel<D, GT><<<grid, kDecThreads, C::kSmemBytes, st>>>(
+        mk, mv, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v),
+        offsets, p.N, num_splits, p.max_splits, p.Hq, p.Hkv, p.scale * kLog2e, part_o, part_ml,
+        device_status_ptr());
   }
   return cudaGetLastError();
 }
@@ -312,23 +388,20 @@ cudaError_t launch_decode_d(const DecodeProblem& p, const void* q, const void* k
   float* part_o = static_cast<float*>(workspace);
   float* part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                             ((slots * D * sizeof(float) + 255) & ~static_cast<size_t>(255)));
+  // K and V as 3-D maps (D, Hkv, rows) over the packed caches. The row extent is nominal (the real
+  // count is on the device); the kernel never issues a box that reaches past kv_offsets[N].
+  CUtensorMap mk, mv;
+  if (!make_map_packed_bf16(&mk, k, kDecMapRows, p.Hkv, D, kDecBlk) ||
+      !make_map_packed_bf16(&mv, v, kDecMapRows, p.Hkv, D, kDecBlk))
+    return cudaErrorInvalidValue;
   const int G = p.Hq / p.Hkv;
   cudaError_t e;
-  bool done = false;
-  if constexpr (D == 64) {  // at D = 128 eight heads per CTA would spill registers
-    if (G % 8 == 0) {
-      e = launch_split<D, 8>(p, q, k, v, offsets, num_splits, part_o, part_ml, st);
-      done = true;
-    }
-  }
-  if (done) {
-  } else if (G % 4 == 0) {
-    e = launch_split<D, 4>(p, q, k, v, offsets, num_splits, part_o, part_ml, st);
-  } else if (G % 2 == 0) {
-    e = launch_split<D, 2>(p, q, k, v, offsets, num_splits, part_o, part_ml, st);
-  } else {
-    e = launch_split<D, 1>(p, q, k, v, offsets, num_splits, part_o, part_ml, st);
-  }
+  if (G % 4 == 0)  // at most four query heads per CTA
+    e = launch_split<D, 4>(p, q, k, v, mk, mv, offsets, num_splits, part_o, part_ml, st);
+  else if (G % 2 == 0)
+    e = launch_split<D, 2>(p, q, k, v, mk, mv, offsets, num_splits, part_o, part_ml, st);
+  else
+    e = launch_split<D, 1>(p, q, k, v, mk, mv, offsets, num_splits, part_o, part_ml, st);
   if (e != cudaSuccess) return e;
   const long long warps = static_cast<long long>(p.N) * p.Hq;
   {

@@ -3,28 +3,33 @@
 // The forward is one reduction over key blocks under the online-softmax monoid ("Não escreva
 // kernels, derive-os", "Aprofundamento", first paragraph): for every query row the CTA keeps the
 // triple (m, l, O) -- running max (base-2 units), running sum of 2^(s - m) and the unnormalised
-// output -- and folds in one 64-key block at a time:
+// output -- and folds in one 128-key block at a time:
 //   S = Q K^T (tensor cores, fp32 in TMEM), m' = max(m, rowmax S), P = 2^(S - m'),
 //   l = l 2^(m - m') + rowsum P, O = O 2^(m - m') + P V (tensor cores, fp32 in TMEM).
-// The two contractions are dense, so they run as tcgen05.mma (bf16 operands from shared memory,
-// fp32 accumulators in tensor memory); the row statistics run on the CUDA cores, one thread per row.
+// The two contractions are dense, so they run as tcgen05.mma with fp32 accumulators in tensor
+// memory; the row statistics run on the CUDA cores, one thread per row.
 //
-// A CTA owns two 128-row query tiles of one head and streams the key/value blocks once for both,
-// which halves the K/V bytes each SM pulls from L2 per tensor-core FLOP (with one tile per CTA
-// the SM's L2 read bandwidth, not the tensor cores, set the pace). Warp roles (320 threads):
-//   warps 0-3 / 4-7  softmax of tile 0 / tile 1: read S from TMEM, mask, row max / sum, write P
-//                    (bf16, swizzled, double-buffered) to SMEM, rescale O in TMEM when a row max
-//                    grows by more than 2^8, epilogue O / l and lse. With two P buffers per tile the
-//                    softmax waits for a PV only when it must rescale O.
-//   warp 8           TMA producer: both Q tiles once, then K and V blocks through a ring.
-//   warp 9           TMEM allocator and MMA issuer (one elected lane): S of block j for both tiles
-//                    (double-buffered in TMEM), then P V of block j - 1 for both tiles, so that the
-//                    tensor cores work on one tile while the other tile's softmax runs.
+// A CTA owns two 128-row query tiles of one head and streams each 128-key K/V block once for both.
+// TMEM holds, per tile, S (128 columns) and O (128 columns): 512 in all. The softmax writes P as
+// bf16 back over the first 64 columns of its own S, and P V reads it from there (A operand in
+// TMEM), so P never goes through shared memory. Every MMA is 128 wide in N, which keeps the tensor
+// pipe fed per instruction issued.
+//
+// Warp roles (320 threads):
+//   warps 0-3 / 4-7  softmax of tile 0 / tile 1, one row per thread: S from TMEM in 32-column
+//                    chunks (row max, then exp2, row sum and P), lazy O rescale, P to TMEM;
+//                    epilogue O / l and lse.
+//   warp 8           TMA producer: both Q tiles once, then K and V blocks through two rings.
+//   warp 9           TMEM allocator and MMA issuer (one elected lane of a converged warp): for each
+//                    tile, O += P V of block j and then at once S = Q K^T of block j + 1, tile 0 and
+//                    tile 1 alternating, so the tensor pipe works on one tile while the other tile's
+//                    softmax runs. MMAs execute in issue order, so once S of block j is complete,
+//                    P V of block j - 1 is too: the softmax may rescale O then without a further wait.
 // Lazy rescaling: a row keeps its old max m while the block max stays within m + 8 (base 2); P then
 // stays <= 256 and the final O / l and lse = m + log2 l use the same m, so the result is exact.
 //
-// Shared-memory tiles use the 128-byte swizzle: Q, K and P are K-major (rows of 64 bf16 = 128 B),
-// V is read as an MN-major operand (its head dim is contiguous). Every wait is bounded (common.cuh).
+// Shared-memory tiles use the 128-byte swizzle: Q and K are K-major (rows of 64 bf16 = 128 B), V is
+// read as an MN-major operand (its head dim is contiguous). Every wait is bounded (common.cuh).
 #include <math.h>
 
 #include "common.cuh"
@@ -35,27 +40,25 @@ namespace attn {
 namespace {
 
 constexpr int kBM = 128;   // query rows per tile (two tiles per CTA)
-constexpr int kBN = 64;    // keys per block
+constexpr int kBN = 128;   // keys per block
 constexpr int kThreads = 320;
-constexpr int kQAtom = 128 * 128;  // 128 rows x 128 bytes (16 KB)
-constexpr int kKAtom = 64 * 128;   // 64 rows x 128 bytes (8 KB)
+constexpr int kAtom = 128 * 128;  // 128 rows x 128 bytes (16 KB)
 
 template <int D>
 struct FwdCfg {
-  static constexpr int kAtoms = D / 64;                  // 64-element column atoms per row
-  static constexpr int kQBytes = kAtoms * kQAtom;        // one 128 x D query tile
-  static constexpr int kKVBytes = kAtoms * kKAtom;       // one 64 x D key or value block
-  static constexpr int kStages = (D == 128) ? 3 : 6;  // 224 KB of tiles at D = 128
-  static constexpr int kOffQ = 0;                                  // [2 tiles]
-  static constexpr int kOffK = kOffQ + 2 * kQBytes;                // [stages]
-  static constexpr int kOffV = kOffK + kStages * kKVBytes;         // [stages]
-  static constexpr int kOffP = kOffV + kStages * kKVBytes;         // [tile][buffer] 128 x 64 bf16 = 16 KB
-  static constexpr int kOffBar = kOffP + 4 * kQAtom;
-  static constexpr int kNumBars = 1 + 4 * kStages + 4 + 4 + 4 + 4 + 1;
+  static constexpr int kAtoms = D / 64;              // 64-element column atoms per row
+  static constexpr int kTileBytes = kAtoms * kAtom;  // one 128 x D tile (Q, K or V)
+  static constexpr int kKStages = (D == 128) ? 2 : 4;
+  static constexpr int kVStages = (D == 128) ? 2 : 4;
+  static constexpr int kOffQ = 0;                                      // [2 tiles]
+  static constexpr int kOffK = kOffQ + 2 * kTileBytes;                 // [K stages]
+  static constexpr int kOffV = kOffK + kKStages * kTileBytes;          // [V stages]
+  static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + slack for 1024-byte alignment
-  // TMEM: S of tile t, buffer u at column 64 * (2t + u); O of tile t at 256 + 128 t.
-  __host__ __device__ static constexpr uint32_t colS(int t, int u) { return 64u * (2 * t + u); }
+  // TMEM: S (and P over its first 64 columns) of tile t at 128 t; O of tile t at 256 + 128 t.
+  __host__ __device__ static constexpr uint32_t colS(int t) { return 128u * t; }
   __host__ __device__ static constexpr uint32_t colO(int t) { return 256u + 128u * t; }
 };
 
@@ -78,7 +81,7 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-// Number of 64-key blocks some row of the 128-row tile starting at `qs` can see.
+// Number of 128-key blocks some row of the 128-row tile starting at `qs` can see.
 __device__ __forceinline__ int tile_blocks(const FwdArgs& a, int qs) {
   if (qs >= a.Sq) return 0;
   int kv_end = a.Sk;
@@ -96,18 +99,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = smem + C::kOffQ;
   uint8_t* sK = smem + C::kOffK;
   uint8_t* sV = smem + C::kOffV;
-  uint8_t* sP = smem + C::kOffP;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = k_full + C::kStages;
-  uint64_t* v_full = k_empty + C::kStages;
-  uint64_t* v_empty = v_full + C::kStages;
-  uint64_t* s_full = v_empty + C::kStages;  // [tile][buffer]
-  uint64_t* s_free = s_full + 4;            // [tile][buffer]
-  uint64_t* p_full = s_free + 4;            // [tile][P buffer]
-  uint64_t* o_done = p_full + 4;            // [tile][P buffer]: the PV that read that P buffer is done
-  uint64_t* drain = o_done + 4;
+  uint64_t* k_empty = k_full + C::kKStages;
+  uint64_t* v_full = k_empty + C::kKStages;
+  uint64_t* v_empty = v_full + C::kVStages;
+  uint64_t* s_full = v_empty + C::kVStages;  // [tile]
+  uint64_t* p_full = s_full + 2;             // [tile]
+  uint64_t* o_done = p_full + 2;             // [tile]: every P V of the tile is complete
+  uint64_t* drain = o_done + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
 
@@ -124,19 +125,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < C::kKStages; ++s) {
       mbar_init(k_full + s, 1);
       mbar_init(k_empty + s, 1);
+    }
+    for (int s = 0; s < C::kVStages; ++s) {
       mbar_init(v_full + s, 1);
       mbar_init(v_empty + s, 1);
     }
-    for (int s = 0; s < 4; ++s) {
-      mbar_init(s_full + s, 1);
-      mbar_init(s_free + s, 4);
-    }
-    for (int s = 0; s < 4; ++s) {
-      mbar_init(p_full + s, 4);
-      mbar_init(o_done + s, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(s_full + t, 1);
+      mbar_init(p_full + t, 4);
+      mbar_init(o_done + t, 1);
     }
     mbar_init(drain, 1);
     *abort = 0;
@@ -159,40 +159,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 8) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0 && nmax > 0) {
-      constexpr uint32_t kQTx = kBM * D * 2;
-      constexpr uint32_t kKVTx = kBN * D * 2;
-      mbar_arrive_expect_tx(q_full, (n0 > 0 ? kQTx : 0u) + (n1 > 0 ? kQTx : 0u));
+      constexpr uint32_t kTx = kBM * D * 2;
+      mbar_arrive_expect_tx(q_full, (n0 > 0 ? kTx : 0u) + (n1 > 0 ? kTx : 0u));
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         if ((t == 0 ? n0 : n1) == 0) continue;
 #pragma unroll
         for (int at = 0; at < C::kAtoms; ++at)
-          tma_load_4d(sQ + t * C::kQBytes + at * kQAtom, &tmQ, q_full, at * 64, h, q0 + t * kBM, b);
+          tma_load_4d(sQ + t * C::kTileBytes + at * kAtom, &tmQ, q_full, at * 64, h, q0 + t * kBM, b);
       }
       int issued_k = 0, issued_v = 0;
       for (int j = 0; j < nmax; ++j) {
-        const int s = j % C::kStages;
-        const uint32_t ph = (j / C::kStages) & 1;
-        if (!mbar_wait(k_empty + s, ph ^ 1, abort, a.status)) break;
-        mbar_arrive_expect_tx(k_full + s, kKVTx);
+        const int sk = j % C::kKStages, sv = j % C::kVStages;
+        if (!mbar_wait(k_empty + sk, ((j / C::kKStages) & 1) ^ 1, abort, a.status)) break;
+        mbar_arrive_expect_tx(k_full + sk, kTx);
 #pragma unroll
         for (int at = 0; at < C::kAtoms; ++at)
-          tma_load_4d(sK + s * C::kKVBytes + at * kKAtom, &tmK, k_full + s, at * 64, g, j * kBN, b);
+          tma_load_4d(sK + sk * C::kTileBytes + at * kAtom, &tmK, k_full + sk, at * 64, g, j * kBN, b);
         issued_k = j + 1;
-        if (!mbar_wait(v_empty + s, ph ^ 1, abort, a.status)) break;
-        mbar_arrive_expect_tx(v_full + s, kKVTx);
+        if (!mbar_wait(v_empty + sv, ((j / C::kVStages) & 1) ^ 1, abort, a.status)) break;
+        mbar_arrive_expect_tx(v_full + sv, kTx);
 #pragma unroll
         for (int at = 0; at < C::kAtoms; ++at)
-          tma_load_4d(sV + s * C::kKVBytes + at * kKAtom, &tmV, v_full + s, at * 64, g, j * kBN, b);
+          tma_load_4d(sV + sv * C::kTileBytes + at * kAtom, &tmV, v_full + sv, at * 64, g, j * kBN, b);
         issued_v = j + 1;
       }
       // Let every load this thread issued land before the CTA can exit. On the normal path the
       // consumers have already waited for each of them, so these return at once.
       wait_drain(q_full, 0);
-      for (int j = max(0, issued_k - C::kStages); j < issued_k; ++j)
-        wait_drain(k_full + j % C::kStages, (j / C::kStages) & 1);
-      for (int j = max(0, issued_v - C::kStages); j < issued_v; ++j)
-        wait_drain(v_full + j % C::kStages, (j / C::kStages) & 1);
+      for (int j = max(0, issued_k - C::kKStages); j < issued_k; ++j)
+        wait_drain(k_full + j % C::kKStages, (j / C::kKStages) & 1);
+      for (int j = max(0, issued_v - C::kVStages); j < issued_v; ++j)
+        wait_drain(v_full + j % C::kVStages, (j / C::kVStages) & 1);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
@@ -202,61 +200,71 @@ __global__ void __launch_bounds__(kThreads, 1)
       // base descriptors, built once; each MMA only moves the start address
       const uint64_t dQ0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);
-      const uint64_t dV0 = sdesc_sw128(smem_u32(sV), kKAtom, 1024);
-      const uint64_t dP0 = sdesc_sw128(smem_u32(sP), 16, 1024);
+      const uint64_t dV0 = sdesc_sw128(smem_u32(sV), kAtom, 1024);
       const int nt[2] = {n0, n1};
       bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort, a.status));
-      for (int j = 0; ok && j <= nmax; ++j) {
-        if (j < nmax) {
-          const int s = j % C::kStages;
-          if (!__all_sync(0xffffffffu, mbar_wait(k_full + s, (j / C::kStages) & 1, abort, a.status))) break;
-          const uint64_t dK = sdesc_advance(dK0, s * C::kKVBytes);
-          for (int t = 0; t < 2; ++t) {
-            if (j >= nt[t]) continue;
-            const int u = j & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(s_free + 2 * t + u, ((j >> 1) & 1) ^ 1, abort, a.status))) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint64_t dQ = sdesc_advance(dQ0, t * C::kQBytes);
-            const uint32_t dS = tmem + C::colS(t, u);
+      int k_ready = -1, v_ready = -1;  // last K / V block this warp has waited for
+      auto wait_k = [&](int jb) -> bool {
+        if (k_ready >= jb) return true;
+        k_ready = jb;
+        return __all_sync(0xffffffffu, mbar_wait(k_full + jb % C::kKStages, (jb / C::kKStages) & 1, abort, a.status)) != 0;
+      };
+      auto wait_v = [&](int jb) -> bool {
+        if (v_ready >= jb) return true;
+        v_ready = jb;
+        return __all_sync(0xffffffffu, mbar_wait(v_full + jb % C::kVStages, (jb / C::kVStages) & 1, abort, a.status)) != 0;
+      };
+      // S_t of block jb = Q_t K_jb^T
+      auto issue_s = [&](int t, int jb) {
+        tc_fence_after();
+        const uint64_t dK = sdesc_advance(dK0, (jb % C::kKStages) * C::kTileBytes);
+        const uint64_t dQ = sdesc_advance(dQ0, t * C::kTileBytes);
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              umma_ss_warp(dS, sdesc_advance(dQ, (kk >> 2) * kQAtom + (kk & 3) * 32),
-                      sdesc_advance(dK, (kk >> 2) * kKAtom + (kk & 3) * 32), kIdescS, kk > 0);
-            }
-            umma_commit_warp(s_full + 2 * t + u);
-          }
-          if (!ok) break;
-          umma_commit_warp(k_empty + s);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
+          umma_ss_warp(tmem + C::colS(t), sdesc_advance(dQ, off), sdesc_advance(dK, off), kIdescS, kk > 0);
         }
-        if (j >= 1) {
-          const int jj = j - 1;
-          const int s = jj % C::kStages;
-          if (!__all_sync(0xffffffffu, mbar_wait(v_full + s, (jj / C::kStages) & 1, abort, a.status))) break;
-          const uint64_t dV = sdesc_advance(dV0, s * C::kKVBytes);
-          for (int t = 0; t < 2; ++t) {
-            if (jj >= nt[t]) continue;
-            const int pb = jj & 1;  // P buffer of block jj
-            if (!__all_sync(0xffffffffu, mbar_wait(p_full + 2 * t + pb, (jj >> 1) & 1, abort, a.status))) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint64_t dP = sdesc_advance(dP0, (2 * t + pb) * kQAtom);
-            const uint32_t dO = tmem + C::colO(t);
-#pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk) {
-              umma_ss_warp(dO, sdesc_advance(dP, kk * 32), sdesc_advance(dV, kk * 16 * 128), kIdescO, (jj > 0 || kk > 0));
-            }
-            umma_commit_warp(o_done + 2 * t + pb);
-          }
-          if (!ok) break;
-          umma_commit_warp(v_empty + s);
-        }
+        umma_commit_warp(s_full + t);
+      };
+      // per block j and tile t: O_t += P_t V_j, then at once S_t of block j + 1 (it overwrites P_t in
+      // TMEM; the P V that reads P_t was issued just before it and MMAs execute in order). The two
+      // tiles' chains are independent, so the tensor pipe alternates between them.
+      if (ok && wait_k(0)) {
+        for (int t = 0; t < 2; ++t)
+          if (nt[t] > 0) issue_s(t, 0);
+        umma_commit_warp(k_empty);
+      } else {
+        ok = false;
       }
-      // all MMAs issued by this thread complete before the CTA releases TMEM
+      for (int j = 0; ok && j < nmax; ++j) {
+        for (int t = 0; t < 2; ++t) {
+          if (j < nt[t]) {
+            if (!wait_v(j) || !__all_sync(0xffffffffu, mbar_wait(p_full + t, j & 1, abort, a.status))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t dV = sdesc_advance(dV0, (j % C::kVStages) * C::kTileBytes);
+            // P (bf16) is the A operand in TMEM, 16 keys = 8 columns per step
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk)
+              umma_ts_warp(tmem + C::colO(t), tmem + C::colS(t) + kk * 8, sdesc_advance(dV, kk * 16 * 128), kIdescO,
+                           (j > 0 || kk > 0));
+            if (j == nt[t] - 1) umma_commit_warp(o_done + t);
+          }
+          if (j + 1 < nt[t]) {
+            if (!wait_k(j + 1)) {
+              ok = false;
+              break;
+            }
+            issue_s(t, j + 1);
+          }
+        }
+        if (!ok) break;
+        if (j + 1 < nmax) umma_commit_warp(k_empty + (j + 1) % C::kKStages);
+        umma_commit_warp(v_empty + j % C::kVStages);
+      }
+      // all MMAs issued by this warp complete before the CTA releases TMEM
       umma_commit_warp(drain);
       wait_drain(drain, 0);
       __syncwarp();
@@ -266,11 +274,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t = warp >> 2;               // query tile of this warpgroup
     const int row = threadIdx.x & 127;     // TMEM lane == row in the tile
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_addr + C::colS(t);
+    const uint32_t tO = tmem + lane_addr + C::colO(t);
     const int n_kv = t == 0 ? n0 : n1;
     const int qrow = q0 + t * kBM + row;
     int row_limit = a.Sk - 1;  // largest visible key index for this row
     if (a.causal) row_limit = min(row_limit, qrow + a.Sk - a.Sq);
-    uint8_t* myP = sP + 2 * t * kQAtom;  // this tile's two P buffers
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     // every lane waits; the outcome is made warp-uniform before any warp-collective tcgen05 op
@@ -279,90 +288,77 @@ __global__ void __launch_bounds__(kThreads, 1)
       return __all_sync(0xffffffffu, r);
     };
     for (int j = 0; j < n_kv; ++j) {
-      const int u = j & 1;
-      if (!wait_warp(s_full + 2 * t + u, (j >> 1) & 1)) {
+      if (!wait_warp(s_full + t, j & 1)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sr[kBN];
-#pragma unroll
-      for (int c = 0; c < kBN / 16; ++c) tmem_ld16(tmem + lane_addr + C::colS(t, u) + c * 16, sr + c * 16);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free + 2 * t + u);
-
       const int kbase = j * kBN;
       const bool need_mask = kbase + kBN - 1 > row_limit;
+      // pass 1: row max, 32 columns at a time (the values are read again in pass 2)
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four independent max chains
+#pragma unroll 1
+      for (int ch = 0; ch < kBN / 32; ++ch) {
+        uint32_t sr[32];
+        tmem_ld16(tS + ch * 32, sr);
+        tmem_ld16(tS + ch * 32 + 16, sr + 16);
+        tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        float x = __uint_as_float(sr[c]) * a.scale_log2;
-        if (need_mask && kbase + c > row_limit) x = -INFINITY;
-        sr[c] = __float_as_uint(x);
-        mx4[c & 3] = fmaxf(mx4[c & 3], x);
+        for (int c = 0; c < 32; ++c) {
+          float x = __uint_as_float(sr[c]);
+          if (need_mask && kbase + ch * 32 + c > row_limit) x = -INFINITY;
+          mx4[c & 3] = fmaxf(mx4[c & 3], x);
+        }
       }
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * a.scale_log2;
       // lazy rescale: move the reference max only when the block max exceeds it by more than 8
       float alpha = 1.f;
       if (mx > m + 8.f || (m == -INFINITY && mx != -INFINITY)) {
         alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - mx);
         m = mx;
       }
-      const float m_use = (m == -INFINITY) ? 0.f : m;
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent sum chains
-      uint32_t pk[kBN / 2];
+      // S of block j is complete, hence so is P V of block j - 1: O may be rescaled now.
+      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 16) {
+          uint32_t orr[16];
+          tmem_ld16(tO + c0, orr);
+          tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < kBN; c += 2) {
-        const float p0 = fast_exp2(__uint_as_float(sr[c]) - m_use);
-        const float p1 = fast_exp2(__uint_as_float(sr[c + 1]) - m_use);
-        rs4[(c >> 1) & 3] += p0 + p1;
-        pk[c / 2] = pack_bf16(p0, p1);
+          for (int e = 0; e < 16; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+          tmem_st16(tO + c0, orr);
+        }
+      }
+      const float m_use = (m == -INFINITY) ? 0.f : m;
+      // pass 2: P = 2^(scale s - m) as bf16 pairs. Chunk ch (keys 32 ch .. 32 ch + 31) goes to columns
+      // 16 ch .. 16 ch + 15, which hold S values already read.
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent sum chains
+#pragma unroll 1
+      for (int ch = 0; ch < kBN / 32; ++ch) {
+        uint32_t sr[32];
+        tmem_ld16(tS + ch * 32, sr);
+        tmem_ld16(tS + ch * 32 + 16, sr + 16);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          float x0 = fmaf(__uint_as_float(sr[c]), a.scale_log2, -m_use);
+          float x1 = fmaf(__uint_as_float(sr[c + 1]), a.scale_log2, -m_use);
+          if (need_mask && kbase + ch * 32 + c > row_limit) x0 = -INFINITY;
+          if (need_mask && kbase + ch * 32 + c + 1 > row_limit) x1 = -INFINITY;
+          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          rs4[(c >> 1) & 3] += p0 + p1;
+          pk[c / 2] = pack_bf16(p0, p1);
+        }
+        tmem_st16(tS + ch * 16, pk);
       }
       l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
-
-      // P buffer j & 1 was last read by the PV of block j - 2: wait for it before overwriting.
-      const int pb = j & 1;
-      if (j >= 2) {
-        if (!wait_warp(o_done + 2 * t + pb, ((j - 2) >> 1) & 1)) {
-          ok = false;
-          break;
-        }
-      }
-      // O may be rescaled only once the PV of block j - 1 has landed (rare with lazy rescaling).
-      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        if (!wait_warp(o_done + 2 * t + (pb ^ 1), ((j - 1) >> 1) & 1)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        {
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 16) {
-            uint32_t orr[16];
-            tmem_ld16(tmem + lane_addr + C::colO(t) + c0, orr);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-            tmem_st16(tmem + lane_addr + C::colO(t) + c0, orr);
-          }
-          tmem_wait_st();
-        }
-      }
-      // P row -> shared memory, 128-byte swizzled K-major (one 64-key atom)
-#pragma unroll
-      for (int ch = 0; ch < kBN / 8; ++ch) {
-        *reinterpret_cast<uint4*>(myP + pb * kQAtom + sw128_offset(row, ch)) =
-            make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-      }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full + 2 * t + pb);
+      if (lane == 0) mbar_arrive(p_full + t);
     }
-    // the last PV of this tile (it was issued after every earlier one)
-    if (ok && n_kv > 0) ok = wait_warp(o_done + 2 * t + ((n_kv - 1) & 1), ((n_kv - 1) >> 1) & 1);
+    if (ok && n_kv > 0) ok = wait_warp(o_done + t, 0);
     tc_fence_after();
     // epilogue: O / l -> bf16, lse = (m + log2 l) ln 2
     const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -372,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c0 = 0; c0 < D; c0 += 16) {
       uint32_t orr[16];
       if (ok && n_kv > 0) {
-        tmem_ld16(tmem + lane_addr + C::colO(t) + c0, orr);
+        tmem_ld16(tO + c0, orr);
         tmem_wait_ld();
       } else {
 #pragma unroll

@@ -46,6 +46,22 @@ inline bool make_map_bshd(CUtensorMap* map, const void* base, CUtensorMapDataTyp
   return r == CUDA_SUCCESS;
 }
 
+// 3-D map over a packed bf16 [rows, H, D] tensor: dims (D, H, rows); boxes of 64 head-dim elements
+// of one head x `box_rows` rows, 128-byte swizzle. `rows` may be a nominal extent: callers must
+// only request boxes that lie inside the real tensor.
+inline bool make_map_packed_bf16(CUtensorMap* map, const void* base, long long rows, int H, int D, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2};
+  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // bf16 [B, S, H, D] with 128-byte swizzle, boxes of 64 head-dim elements x `rows` positions.
 inline bool make_map_bf16_sw128(CUtensorMap* map, const void* base, int B, int S, int H, int D, int rows) {
   return make_map_bshd(map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, S, H, D, 64, rows,

@@ -58,6 +58,10 @@ __device__ __forceinline__ int stream_splits(const int* num_splits, int n, int L
 
 constexpr int kDecBlk = 32;              // keys per block (one per lane)
 constexpr int kDecStages = 4;
+// Compute warp w consumes blocks w, w + 4, ... and every stage has a single-arrival "empty" barrier,
+// so a stage must always belong to the same warp: the stage count is a multiple of the four compute
+// warps (otherwise two warps would share a stage and a parity wait could match the wrong phase).
+static_assert(kDecStages % 4 == 0, "decode ring stages must be a multiple of the compute warps");
 constexpr int kDecThreads = 160;          // four compute warps + one producer warp
 constexpr int kDecMapRows = 0x7fffffff;   // nominal row extent of the K/V tensor maps
 

@@ -16,20 +16,23 @@
 //
 // The main kernel works on transposed score tiles so that keys sit on the TMEM lanes:
 //   S^T = K Q^T and dP^T = V dO^T            (M = 128 keys, N = 128 query rows, K = D).
-// One thread per key computes P^T = 2^(S^T scale log2e - lse2) and dS^T = P^T (dP^T - Delta) and
-// writes both back as bf16 over the first 64 columns of their own TMEM tiles; dS^T also goes to
-// shared memory (128-byte swizzle). Then
-//   dV += P^T dO,  dK += dS^T Q              (A = P^T / dS^T in TMEM, B = dO / Q MN-major in SMEM)
+// One thread per key computes P^T = 2^(S^T scale log2e - lse2) as soon as S^T is in TMEM, and
+// dS^T = P^T (dP^T - Delta) once dP^T is; each is written back as bf16 over the first 64 columns of
+// its own TMEM tile, and dS^T also goes to shared memory (128-byte swizzle). Then
+//   dK += dS^T Q,  dV += P^T dO              (A = dS^T / P^T in TMEM, B = Q / dO MN-major in SMEM)
 //   dQ^T = K^T dS^T                          (M = D, N = 128 query rows, K = 128 keys; both in SMEM)
-// with dQ^T written over the S^T columns. Every MMA is 128 wide in N. MMAs execute in issue order,
-// which is what makes each overwrite in TMEM safe: dV reads P^T before dQ^T overwrites it, dK reads
-// dS^T before the next dP^T overwrites it. For D = 64 the dQ^T MMA still runs with M = 128; the upper
-// 64 TMEM lanes hold values that are never read.
-// TMEM columns: S^T / P^T / dQ^T [0,128), dP^T / dS^T [128,256), dV [256,256+D), dK [384,384+D).
+// with dQ^T written over the dP^T columns, and at once S^T of the next tile over the S^T columns,
+// so that the next tile's scores start while dQ^T is drained; the next dP^T waits for the drain.
+// Every MMA is 128 wide in N. MMAs execute in issue order, which is what makes each overwrite in
+// TMEM safe: dK reads dS^T before dQ^T overwrites it, dV reads P^T before the next S^T does.
+// For D = 64 the dQ^T MMA still runs with M = 128; the upper 64 TMEM lanes hold values that are
+// never read.
+// TMEM columns: S^T / P^T [0,128), dP^T / dS^T / dQ^T [128,256), dV [256,256+D), dK [384,384+D).
 //
 // Warp roles (320 threads): warps 0-3 scores (one key row per thread; at the end the dK/dV
-// epilogue), warps 4-7 dQ drain (one TMEM lane = one head-dim column per thread: tcgen05.ld, then
-// coalesced fp32 reductions into the accumulator, 32 consecutive columns per warp instruction),
+// epilogue), warps 4-7 dQ drain (one TMEM lane = one head-dim column per thread: the whole dQ^T
+// row in one tcgen05.ld, TMEM released at once, then coalesced fp32 reductions into the
+// accumulator, 32 consecutive columns per warp instruction),
 // warp 8 TMA producer (K, V once; Q and dO tiles through a 2-stage ring), warp 9 TMEM allocator
 // and MMA issuer (one elected lane of a converged warp). Every wait is bounded.
 #include <math.h>
@@ -57,7 +60,7 @@ struct BwdCfg {
   static constexpr int kOffDO = kOffQ + kStages * kTileBytes;
   static constexpr int kOffDS = kOffDO + kStages * kTileBytes;  // 128 keys x 128 rows bf16 = 2 atoms
   static constexpr int kOffBar = kOffDS + 2 * kAtom;
-  static constexpr int kNumBars = 1 + 2 * kStages + 8;
+  static constexpr int kNumBars = 1 + 2 * kStages + 9;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
@@ -105,8 +108,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* kv_full = bars;
   uint64_t* q_full = bars + 1;
   uint64_t* q_empty = q_full + C::kStages;
-  uint64_t* s_full = q_empty + C::kStages;  // S^T and dP^T of a tile are in TMEM
-  uint64_t* p_full = s_full + 1;            // P^T, dS^T written (TMEM and shared)
+  uint64_t* s_full = q_empty + C::kStages;  // S^T of a tile is in TMEM
+  uint64_t* dp_full = s_full + 1;           // dP^T of a tile is in TMEM
+  uint64_t* p_full = dp_full + 1;           // P^T, dS^T written (TMEM and shared)
   uint64_t* ds_free = p_full + 1;           // dQ^T MMA done reading dS^T in shared memory
   uint64_t* dq_full = ds_free + 1;          // dQ^T of a tile is in TMEM
   uint64_t* dq_free = dq_full + 1;          // the drain has read dQ^T out of TMEM
@@ -137,6 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(q_empty + s, 1);
     }
     mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
     mbar_init(p_full, 4);
     mbar_init(ds_free, 1);
     mbar_init(dq_full, 1);
@@ -207,48 +212,65 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
         return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, a.status)) != 0;
       };
-      bool ok = wait(kv_full, 0);
+      // S^T (into the S^T columns) and dP^T (into the dP^T columns) of tile jt
+      auto issue_s = [&](int jt) {
+        const uint64_t q = sdesc_advance(kQ, (jt % C::kStages) * C::kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
+          umma_ss_warp(tmem + C::kColS, sdesc_advance(kK, off), sdesc_advance(q, off), kIdS, kk > 0);
+        }
+        umma_commit_warp(s_full);
+      };
+      auto issue_dp = [&](int jt) {
+        const uint64_t dO = sdesc_advance(kDO, (jt % C::kStages) * C::kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
+          umma_ss_warp(tmem + C::kColDP, sdesc_advance(kV, off), sdesc_advance(dO, off), kIdS, kk > 0);
+        }
+        umma_commit_warp(dp_full);
+      };
+      bool ok = wait(kv_full, 0) && wait(q_full, 0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        issue_dp(0);
+      }
       for (int j = 0; ok && j < n_it; ++j) {
         const int s = j % C::kStages;
-        // S^T and dP^T of tile j. S^T overwrites the dQ^T of tile j - 1: the drain must have read it.
-        if (!wait(q_full + s, (j / C::kStages) & 1) || !wait(dq_free, (j & 1) ^ 1)) break;
-        tc_fence_after();
-        {
-          const uint64_t q = sdesc_advance(kQ, s * C::kTileBytes), dO = sdesc_advance(kDO, s * C::kTileBytes);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
-            umma_ss_warp(tmem + C::kColS, sdesc_advance(kK, off), sdesc_advance(q, off), kIdS, kk > 0);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
-            umma_ss_warp(tmem + C::kColDP, sdesc_advance(kV, off), sdesc_advance(dO, off), kIdS, kk > 0);
-          }
-          umma_commit_warp(s_full);
-        }
         // gradients of tile j once P^T and dS^T are written
         if (!wait(p_full, j & 1)) break;
         tc_fence_after();
         {
           const uint64_t q = sdesc_advance(mQ, s * C::kTileBytes), dO = sdesc_advance(mDO, s * C::kTileBytes);
-          // dV += P^T dO and dK += dS^T Q: K = 128 query rows in 8 steps of 16 (8 TMEM columns each)
-#pragma unroll
-          for (int kk = 0; kk < kBM / 16; ++kk)
-            umma_ts_warp(tmem + C::kColDV, tmem + C::kColS + kk * 8, sdesc_advance(dO, kk * 16 * 128), kIdG,
-                         (j > 0 || kk > 0));
+          // dK += dS^T Q and dV += P^T dO: K = 128 query rows in 8 steps of 16 (8 TMEM columns each)
 #pragma unroll
           for (int kk = 0; kk < kBM / 16; ++kk)
             umma_ts_warp(tmem + C::kColDK, tmem + C::kColDP + kk * 8, sdesc_advance(q, kk * 16 * 128), kIdG,
                          (j > 0 || kk > 0));
-          // dQ^T = K^T dS^T over the S^T / P^T columns: K = 128 keys in 8 steps of 16
+#pragma unroll
+          for (int kk = 0; kk < kBM / 16; ++kk)
+            umma_ts_warp(tmem + C::kColDV, tmem + C::kColS + kk * 8, sdesc_advance(dO, kk * 16 * 128), kIdG,
+                         (j > 0 || kk > 0));
+          // dQ^T = K^T dS^T over the dP^T / dS^T columns (dK has read dS^T): K = 128 keys, 8 steps of 16
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
-            umma_ss_warp(tmem + C::kColS, sdesc_advance(mK, kk * 16 * 128), sdesc_advance(mDS, kk * 16 * 128), kIdQ,
+            umma_ss_warp(tmem + C::kColDP, sdesc_advance(mK, kk * 16 * 128), sdesc_advance(mDS, kk * 16 * 128), kIdQ,
                          kk > 0);
           umma_commit_warp(q_empty + s);
           umma_commit_warp(ds_free);
           umma_commit_warp(dq_full);
+        }
+        if (j + 1 < n_it) {
+          // S^T of tile j + 1 over P^T of tile j (dV, issued above, reads it first)
+          if (!wait(q_full + (j + 1) % C::kStages, ((j + 1) / C::kStages) & 1)) break;
+          tc_fence_after();
+          issue_s(j + 1);
+          // dP^T of tile j + 1 over dQ^T of tile j: the drain must have read it
+          if (!wait(dq_free, j & 1)) break;
+          tc_fence_after();
+          issue_dp(j + 1);
         }
       }
       umma_commit_warp(all_done);
@@ -281,46 +303,72 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
         break;
       }
+      tc_fence_after();
+      // P^T = 2^(S^T scale log2e - lse2) in two halves of 64 query columns, as bf16 pairs over the
+      // first 64 S^T columns (already read), where the dV MMA and the dS^T step below read them
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t sr[64], pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 16) tmem_ld16(tS + hf * 64 + c, sr + c);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c4 = 0; c4 < 64; c4 += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + hf * 64 + c4);  // same for every lane
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+          for (int e = 0; e < 4; e += 2) {
+            const int c = hf * 64 + c4 + e;
+            float p0 = fast_exp2(fmaf(__uint_as_float(sr[c4 + e]), a.scale_log2, -lv[e]));
+            float p1 = fast_exp2(fmaf(__uint_as_float(sr[c4 + e + 1]), a.scale_log2, -lv[e + 1]));
+            p0 = (c >= cmin && c < cmax) ? p0 : 0.f;
+            p1 = (c + 1 >= cmin && c + 1 < cmax) ? p1 : 0.f;
+            pk[(c4 + e) / 2] = pack_bf16(p0, p1);
+          }
+        }
+        tmem_st16(tS + hf * 32, pk);
+        tmem_st16(tS + hf * 32 + 16, pk + 16);
+      }
+      if (!wait_warp(dp_full, j & 1)) {
+        ok = false;
+        break;
+      }
       // shared dS^T of the previous tile must have been consumed by its dQ^T MMA
       if (!wait_warp(ds_free, (j & 1) ^ 1)) {
         ok = false;
         break;
       }
+      tmem_wait_st();  // this thread's P^T stores are visible to its own loads below
       tc_fence_after();
-#pragma unroll 1
-      for (int ch = 0; ch < kBM / 32; ++ch) {  // 32 query columns at a time
-        uint32_t sr[32], dp[32];
-        tmem_ld16(tS + ch * 32, sr);
-        tmem_ld16(tS + ch * 32 + 16, sr + 16);
-        tmem_ld16(tDP + ch * 32, dp);
-        tmem_ld16(tDP + ch * 32 + 16, dp + 16);
-        tmem_wait_ld();
-        uint32_t pk[16], dk[16];
+      // dS^T = P^T (dP^T - Delta), from the bf16 P^T above, in two halves of 64 query columns
 #pragma unroll
-        for (int c4 = 0; c4 < 32; c4 += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + ch * 32 + c4);  // same for every lane
-          const float4 d4 = *reinterpret_cast<const float4*>(dlt + ch * 32 + c4);
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t dp[64], pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 16) tmem_ld16(tDP + hf * 64 + c, dp + c);
+        tmem_ld16(tS + hf * 32, pk);
+        tmem_ld16(tS + hf * 32 + 16, pk + 16);
+        tmem_wait_ld();
+        uint32_t dk[32];
+#pragma unroll
+        for (int c4 = 0; c4 < 64; c4 += 4) {
+          const float4 d4 = *reinterpret_cast<const float4*>(dlt + hf * 64 + c4);
+          const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
           for (int e = 0; e < 4; e += 2) {
-            const int c = ch * 32 + c4 + e;
-            float p0 = fast_exp2(fmaf(__uint_as_float(sr[c4 + e]), a.scale_log2, -lv[e]));
-            float p1 = fast_exp2(fmaf(__uint_as_float(sr[c4 + e + 1]), a.scale_log2, -lv[e + 1]));
-            p0 = (c >= cmin && c < cmax) ? p0 : 0.f;
-            p1 = (c + 1 >= cmin && c + 1 < cmax) ? p1 : 0.f;
-            const float d0 = p0 * (__uint_as_float(dp[c4 + e]) - dv4[e]);
-            const float d1 = p1 * (__uint_as_float(dp[c4 + e + 1]) - dv4[e + 1]);
-            pk[(c4 + e) / 2] = pack_bf16(p0, p1);
+            const uint32_t pw = pk[(c4 + e) / 2];
+            const float d0 = bf16_lo(pw) * (__uint_as_float(dp[c4 + e]) - dv4[e]);
+            const float d1 = bf16_hi(pw) * (__uint_as_float(dp[c4 + e + 1]) - dv4[e + 1]);
             dk[(c4 + e) / 2] = pack_bf16(d0, d1);
           }
         }
-        // P^T and dS^T over columns 16 ch .. 16 ch + 15 of their own tiles (already read), and dS^T
-        // to shared memory: key row t, query columns 32 ch .. 32 ch + 31 (atom ch / 2, chunks 4 (ch & 1) ..)
-        tmem_st16(tS + ch * 16, pk);
-        tmem_st16(tDP + ch * 16, dk);
+        // dS^T over dP^T columns 32 hf .. 32 hf + 31 (already read), and to shared memory: key row
+        // t, query columns 64 hf .. 64 hf + 63 = swizzle atom hf
+        tmem_st16(tDP + hf * 32, dk);
+        tmem_st16(tDP + hf * 32 + 16, dk + 16);
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          *reinterpret_cast<uint4*>(sDS + (ch >> 1) * kAtom + sw128_offset(t, (ch & 1) * 4 + u)) =
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<uint4*>(sDS + hf * kAtom + sw128_offset(t, u)) =
               make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
       }
       tmem_wait_st();
@@ -371,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = warp - 4;
     const int d = wq * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tQ = tmem + lane_addr + C::kColS;
+    const uint32_t tQ = tmem + lane_addr + C::kColDP;
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
       const bool r = mbar_wait(bar, parity, abort, a.status);
       return __all_sync(0xffffffffu, r);
@@ -383,20 +431,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!wait_warp(dq_full, j & 1)) break;
       tc_fence_after();
       float* acc = a.dq_acc + ((static_cast<long long>(b) * a.Sq_pad + q0) * a.Hq + h) * D + d;
-#pragma unroll 1
-      for (int ch = 0; ch < kBM / 32; ++ch) {  // 32 query rows at a time
-        uint32_t r[32];
-        tmem_ld16(tQ + ch * 32, r);
-        tmem_ld16(tQ + ch * 32 + 16, r + 16);
-        tmem_wait_ld();
-        if (ch == kBM / 32 - 1) {  // all of dQ^T has left TMEM: its columns may be reused
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(dq_free);
-        }
-        if (d < D) {  // at D = 64 warps 6 and 7 hold no dQ column
+      // the whole dQ^T row of this lane in one round trip; then its columns may be reused at once
+      uint32_t r[kBM];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) red_add_f32(acc + (ch * 32 + c) * row_stride, __uint_as_float(r[c]));
+      for (int c = 0; c < kBM; c += 16) tmem_ld16(tQ + c, r + c);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_free);
+      if (d < D) {  // at D = 64 warps 6 and 7 hold no dQ column
+#pragma unroll
+        for (int c = 0; c < kBM; ++c) {  // a running pointer: one 64-bit add per row, no address table
+          red_add_f32(acc, __uint_as_float(r[c]));
+          acc += row_stride;
         }
       }
     }

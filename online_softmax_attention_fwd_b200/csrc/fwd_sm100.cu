@@ -294,30 +294,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const int kbase = j * kBN;
-      const bool need_mask = kbase + kBN - 1 > row_limit;
-      // pass 1: row max, 32 columns at a time (the values are read again in pass 2)
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four independent max chains
-#pragma unroll 1
-      for (int ch = 0; ch < kBN / 32; ++ch) {
-        uint32_t sr[32];
-        tmem_ld16(tS + ch * 32, sr);
-        tmem_ld16(tS + ch * 32 + 16, sr + 16);
-        tmem_wait_ld();
+      // the whole 128-column row of S in registers: one round trip to TMEM
+      uint32_t sr[kBN];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          float x = __uint_as_float(sr[c]);
-          if (need_mask && kbase + ch * 32 + c > row_limit) x = -INFINITY;
-          mx4[c & 3] = fmaxf(mx4[c & 3], x);
-        }
+      for (int c = 0; c < kBN; c += 16) tmem_ld16(tS + c, sr + c);
+      tmem_wait_ld();
+      if (kbase + kBN - 1 > row_limit) {  // the block crosses this row's last visible key
+#pragma unroll
+        for (int c = 0; c < kBN; ++c)
+          if (kbase + c > row_limit) sr[c] = __float_as_uint(-INFINITY);
       }
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * a.scale_log2;
+      float mx8[8];  // eight independent max chains
+#pragma unroll
+      for (int c = 0; c < 8; ++c) mx8[c] = __uint_as_float(sr[c]);
+#pragma unroll
+      for (int c = 8; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+                       a.scale_log2;
       // lazy rescale: move the reference max only when the block max exceeds it by more than 8
       float alpha = 1.f;
       if (mx > m + 8.f || (m == -INFINITY && mx != -INFINITY)) {
         alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - mx);
         m = mx;
       }
-      // S of block j is complete, hence so is P V of block j - 1: O may be rescaled now.
+      const float m_use = (m == -INFINITY) ? 0.f : m;
+      // P = 2^(scale s - m) as bf16 pairs over the first 64 columns of S
+      float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // eight independent sum chains
+      uint32_t pk[kBN / 2];
+#pragma unroll
+      for (int c = 0; c < kBN; c += 2) {
+        const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c]), a.scale_log2, -m_use));
+        const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), a.scale_log2, -m_use));
+        rs8[(c >> 1) & 7] += p0 + p1;
+        pk[c / 2] = pack_bf16(p0, p1);
+      }
+#pragma unroll
+      for (int c = 0; c < kBN / 2; c += 16) tmem_st16(tS + c, pk + c);
+      // S of block j is complete, hence so is P V of block j - 1: O may be rescaled now, before
+      // P V of block j is released below.
       if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 16) {
@@ -329,30 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st16(tO + c0, orr);
         }
       }
-      const float m_use = (m == -INFINITY) ? 0.f : m;
-      // pass 2: P = 2^(scale s - m) as bf16 pairs. Chunk ch (keys 32 ch .. 32 ch + 31) goes to columns
-      // 16 ch .. 16 ch + 15, which hold S values already read.
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent sum chains
-#pragma unroll 1
-      for (int ch = 0; ch < kBN / 32; ++ch) {
-        uint32_t sr[32];
-        tmem_ld16(tS + ch * 32, sr);
-        tmem_ld16(tS + ch * 32 + 16, sr + 16);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float x0 = fmaf(__uint_as_float(sr[c]), a.scale_log2, -m_use);
-          float x1 = fmaf(__uint_as_float(sr[c + 1]), a.scale_log2, -m_use);
-          if (need_mask && kbase + ch * 32 + c > row_limit) x0 = -INFINITY;
-          if (need_mask && kbase + ch * 32 + c + 1 > row_limit) x1 = -INFINITY;
-          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-          rs4[(c >> 1) & 3] += p0 + p1;
-          pk[c / 2] = pack_bf16(p0, p1);
-        }
-        tmem_st16(tS + ch * 16, pk);
-      }
-      l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
+      l = l * alpha + (((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7])));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();

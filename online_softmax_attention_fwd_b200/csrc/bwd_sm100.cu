@@ -19,14 +19,15 @@
 // One thread per key computes P^T = 2^(S^T scale log2e - lse2) as soon as S^T is in TMEM, and
 // dS^T = P^T (dP^T - Delta) once dP^T is; each is written back as bf16 over the first 64 columns of
 // its own TMEM tile, and dS^T also goes to shared memory (128-byte swizzle). Then
-//   dK += dS^T Q,  dV += P^T dO              (A = dS^T / P^T in TMEM, B = Q / dO MN-major in SMEM)
+//   dV += P^T dO,  dK += dS^T Q              (A = P^T / dS^T in TMEM, B = dO / Q MN-major in SMEM)
 //   dQ^T = K^T dS^T                          (M = D, N = 128 query rows, K = 128 keys; both in SMEM)
-// with dQ^T written over the dP^T columns, and at once S^T of the next tile over the S^T columns,
-// so that the next tile's scores start while dQ^T is drained; the next dP^T waits for the drain.
-// Every MMA is 128 wide in N. MMAs execute in issue order, which is what makes each overwrite in
-// TMEM safe: dK reads dS^T before dQ^T overwrites it, dV reads P^T before the next S^T does.
-// For D = 64 the dQ^T MMA still runs with M = 128; the upper 64 TMEM lanes hold values that are
-// never read.
+// with S^T of the next tile issued right after dV (over P^T, which dV has read), so the next tile's
+// P^T is computed while dK and dQ^T of this tile run; dQ^T goes over the dP^T columns once dK has
+// read dS^T, and the next dP^T waits until the drain has read dQ^T. MMAs execute in issue order,
+// which is what makes each overwrite in TMEM safe. dQ is produced transposed (head dim on the TMEM
+// lanes) so that the drain's reductions are coalesced: a warp adds 32 consecutive head-dim columns
+// of one query row per instruction. For D = 64 the dQ^T MMA still runs with M = 128; the upper 64
+// TMEM lanes hold values that are never read.
 // TMEM columns: S^T / P^T [0,128), dP^T / dS^T / dQ^T [128,256), dV [256,256+D), dK [384,384+D).
 //
 // Warp roles (320 threads): warps 0-3 scores (one key row per thread; at the end the dK/dV
@@ -62,7 +63,8 @@ struct BwdCfg {
   static constexpr int kOffBar = kOffDS + 2 * kAtom;
   static constexpr int kNumBars = 1 + 2 * kStages + 9;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
+  static constexpr int kOffRow = kOffMisc + 64;              // lse2 and Delta of the current tile
+  static constexpr int kSmemBytes = kOffRow + 2 * kBM * 4 + 1024;
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
 };
 
@@ -118,6 +120,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = all_done + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
+  float* sLse = reinterpret_cast<float*>(smem + C::kOffRow);  // [kBM]
+  float* sDlt = sLse + kBM;                                    // [kBM]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = static_cast<int>(blockIdx.x) % a.Hkv;
@@ -239,35 +243,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int j = 0; ok && j < n_it; ++j) {
         const int s = j % C::kStages;
+        const bool more = j + 1 < n_it;
         // gradients of tile j once P^T and dS^T are written
         if (!wait(p_full, j & 1)) break;
         tc_fence_after();
-        {
-          const uint64_t q = sdesc_advance(mQ, s * C::kTileBytes), dO = sdesc_advance(mDO, s * C::kTileBytes);
-          // dK += dS^T Q and dV += P^T dO: K = 128 query rows in 8 steps of 16 (8 TMEM columns each)
+        const uint64_t q = sdesc_advance(mQ, s * C::kTileBytes), dO = sdesc_advance(mDO, s * C::kTileBytes);
+        // dV += P^T dO: K = 128 query rows in 8 steps of 16 (8 TMEM columns each)
 #pragma unroll
-          for (int kk = 0; kk < kBM / 16; ++kk)
-            umma_ts_warp(tmem + C::kColDK, tmem + C::kColDP + kk * 8, sdesc_advance(q, kk * 16 * 128), kIdG,
-                         (j > 0 || kk > 0));
-#pragma unroll
-          for (int kk = 0; kk < kBM / 16; ++kk)
-            umma_ts_warp(tmem + C::kColDV, tmem + C::kColS + kk * 8, sdesc_advance(dO, kk * 16 * 128), kIdG,
-                         (j > 0 || kk > 0));
-          // dQ^T = K^T dS^T over the dP^T / dS^T columns (dK has read dS^T): K = 128 keys, 8 steps of 16
-#pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            umma_ss_warp(tmem + C::kColDP, sdesc_advance(mK, kk * 16 * 128), sdesc_advance(mDS, kk * 16 * 128), kIdQ,
-                         kk > 0);
-          umma_commit_warp(q_empty + s);
-          umma_commit_warp(ds_free);
-          umma_commit_warp(dq_full);
-        }
-        if (j + 1 < n_it) {
-          // S^T of tile j + 1 over P^T of tile j (dV, issued above, reads it first)
+        for (int kk = 0; kk < kBM / 16; ++kk)
+          umma_ts_warp(tmem + C::kColDV, tmem + C::kColS + kk * 8, sdesc_advance(dO, kk * 16 * 128), kIdG,
+                       (j > 0 || kk > 0));
+        // S^T of tile j + 1 over P^T of tile j, which dV has just read: the next tile's P^T can be
+        // computed while dK and dQ^T of this tile run
+        if (more) {
           if (!wait(q_full + (j + 1) % C::kStages, ((j + 1) / C::kStages) & 1)) break;
           tc_fence_after();
           issue_s(j + 1);
-          // dP^T of tile j + 1 over dQ^T of tile j: the drain must have read it
+        }
+        // dK += dS^T Q
+#pragma unroll
+        for (int kk = 0; kk < kBM / 16; ++kk)
+          umma_ts_warp(tmem + C::kColDK, tmem + C::kColDP + kk * 8, sdesc_advance(q, kk * 16 * 128), kIdG,
+                       (j > 0 || kk > 0));
+        // dQ^T = K^T dS^T over the dP^T / dS^T columns (dK has read dS^T): K = 128 keys, 8 steps of 16
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          umma_ss_warp(tmem + C::kColDP, sdesc_advance(mK, kk * 16 * 128), sdesc_advance(mDS, kk * 16 * 128), kIdQ,
+                       kk > 0);
+        umma_commit_warp(q_empty + s);
+        umma_commit_warp(ds_free);
+        umma_commit_warp(dq_full);
+        // dP^T of tile j + 1 over dQ^T of tile j: the drain must have read it
+        if (more) {
           if (!wait(dq_free, j & 1)) break;
           tc_fence_after();
           issue_dp(j + 1);
@@ -299,9 +306,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       // lse2 = +inf, so their P is 0 without a mask.
       const int cmin = a.causal ? key - (a.Sk - a.Sq) - q0 : 0;
       const int cmax = key < a.Sk ? kBM : 0;
+      const bool unmasked = __all_sync(0xffffffffu, cmin <= 0 && cmax == kBM) != 0;
+      // this tile's lse2 and Delta into shared memory, once every score warp is done with the last
+      // tile's; the loads overlap the wait for S^T. Every score warp runs all n_it iterations (one
+      // whose wait failed only passes the barriers), so the named barriers always complete.
+      named_barrier(1, 128);
+      if (ok) {
+        sLse[t] = lse2[t];
+        sDlt[t] = dlt[t];
+      }
+      named_barrier(1, 128);
+      if (!ok) continue;
       if (!wait_warp(s_full, j & 1)) {
         ok = false;
-        break;
+        continue;
       }
       tc_fence_after();
       // P^T = 2^(S^T scale log2e - lse2) in two halves of 64 query columns, as bf16 pairs over the
@@ -314,15 +332,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
 #pragma unroll
         for (int c4 = 0; c4 < 64; c4 += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + hf * 64 + c4);  // same for every lane
+          const float4 l4 = *reinterpret_cast<const float4*>(sLse + hf * 64 + c4);  // same for every lane
           const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
           for (int e = 0; e < 4; e += 2) {
             const int c = hf * 64 + c4 + e;
             float p0 = fast_exp2(fmaf(__uint_as_float(sr[c4 + e]), a.scale_log2, -lv[e]));
             float p1 = fast_exp2(fmaf(__uint_as_float(sr[c4 + e + 1]), a.scale_log2, -lv[e + 1]));
-            p0 = (c >= cmin && c < cmax) ? p0 : 0.f;
-            p1 = (c + 1 >= cmin && c + 1 < cmax) ? p1 : 0.f;
+            if (!unmasked) {
+              p0 = (c >= cmin && c < cmax) ? p0 : 0.f;
+              p1 = (c + 1 >= cmin && c + 1 < cmax) ? p1 : 0.f;
+            }
             pk[(c4 + e) / 2] = pack_bf16(p0, p1);
           }
         }
@@ -331,12 +351,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!wait_warp(dp_full, j & 1)) {
         ok = false;
-        break;
+        continue;
       }
       // shared dS^T of the previous tile must have been consumed by its dQ^T MMA
       if (!wait_warp(ds_free, (j & 1) ^ 1)) {
         ok = false;
-        break;
+        continue;
       }
       tmem_wait_st();  // this thread's P^T stores are visible to its own loads below
       tc_fence_after();
@@ -352,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t dk[32];
 #pragma unroll
         for (int c4 = 0; c4 < 64; c4 += 4) {
-          const float4 d4 = *reinterpret_cast<const float4*>(dlt + hf * 64 + c4);
+          const float4 d4 = *reinterpret_cast<const float4*>(sDlt + hf * 64 + c4);
           const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
           for (int e = 0; e < 4; e += 2) {
@@ -430,7 +450,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int q0 = (qt0 + j % n_q) * kBM;
       if (!wait_warp(dq_full, j & 1)) break;
       tc_fence_after();
-      float* acc = a.dq_acc + ((static_cast<long long>(b) * a.Sq_pad + q0) * a.Hq + h) * D + d;
       // the whole dQ^T row of this lane in one round trip; then its columns may be reused at once
       uint32_t r[kBM];
 #pragma unroll
@@ -440,6 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_free);
       if (d < D) {  // at D = 64 warps 6 and 7 hold no dQ column
+        float* acc = a.dq_acc + ((static_cast<long long>(b) * a.Sq_pad + q0) * a.Hq + h) * D + d;
 #pragma unroll
         for (int c = 0; c < kBM; ++c) {  // a running pointer: one 64-bit add per row, no address table
           red_add_f32(acc, __uint_as_float(r[c]));

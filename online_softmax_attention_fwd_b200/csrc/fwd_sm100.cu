@@ -42,6 +42,12 @@ namespace {
 constexpr int kBM = 128;   // query rows per tile (two tiles per CTA)
 constexpr int kBN = 128;   // keys per block
 constexpr int kThreads = 320;
+// Eighths of each unmasked block's exponentials computed on the FMA pipe instead of ex2 (the
+// transcendental unit is the softmax's bottleneck).
+#ifndef ATTN_FWD_POLY_EIGHTHS
+#define ATTN_FWD_POLY_EIGHTHS 0
+#endif
+constexpr int kPolyEighths = ATTN_FWD_POLY_EIGHTHS;
 constexpr int kAtom = 128 * 128;  // 128 rows x 128 bytes (16 KB)
 
 template <int D>
@@ -54,7 +60,7 @@ struct FwdCfg {
   static constexpr int kOffK = kOffQ + 2 * kTileBytes;                 // [K stages]
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;          // [V stages]
   static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
-  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1;
+  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 4 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + slack for 1024-byte alignment
   // TMEM: S (and P over its first 64 columns) of tile t at 128 t; O of tile t at 256 + 128 t.
@@ -106,8 +112,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_full = k_empty + C::kKStages;
   uint64_t* v_empty = v_full + C::kVStages;
   uint64_t* s_full = v_empty + C::kVStages;  // [tile]
-  uint64_t* p_full = s_full + 2;             // [tile]
-  uint64_t* o_done = p_full + 2;             // [tile]: every P V of the tile is complete
+  uint64_t* p_full = s_full + 2;             // [tile][half]: P of keys 0-63 / 64-127 in TMEM
+  uint64_t* o_done = p_full + 4;             // [tile]: every P V of the tile is complete
   uint64_t* drain = o_done + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
@@ -135,7 +141,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(s_full + t, 1);
-      mbar_init(p_full + t, 4);
+      mbar_init(p_full + 2 * t, 4);
+      mbar_init(p_full + 2 * t + 1, 4);
       mbar_init(o_done + t, 1);
     }
     mbar_init(drain, 1);
@@ -239,17 +246,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; ok && j < nmax; ++j) {
         for (int t = 0; t < 2; ++t) {
           if (j < nt[t]) {
-            if (!wait_v(j) || !__all_sync(0xffffffffu, mbar_wait(p_full + t, j & 1, abort, a.status))) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
             const uint64_t dV = sdesc_advance(dV0, (j % C::kVStages) * C::kTileBytes);
-            // P (bf16) is the A operand in TMEM, 16 keys = 8 columns per step
+            // P (bf16) is the A operand in TMEM, 16 keys = 8 columns per step; each half of the
+            // block's keys goes as soon as the softmax has written its P
 #pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk)
-              umma_ts_warp(tmem + C::colO(t), tmem + C::colS(t) + kk * 8, sdesc_advance(dV, kk * 16 * 128), kIdescO,
-                           (j > 0 || kk > 0));
+            for (int hf = 0; hf < 2; ++hf) {
+              if ((hf == 0 && !wait_v(j)) ||
+                  !__all_sync(0xffffffffu, mbar_wait(p_full + 2 * t + hf, j & 1, abort, a.status))) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 4 * hf; kk < 4 * hf + 4; ++kk)
+                umma_ts_warp(tmem + C::colO(t), tmem + C::colS(t) + kk * 8, sdesc_advance(dV, kk * 16 * 128),
+                             kIdescO, (j > 0 || kk > 0));
+            }
+            if (!ok) break;
             if (j == nt[t] - 1) umma_commit_warp(o_done + t);
           }
           if (j + 1 < nt[t]) {
@@ -319,36 +332,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = mx;
       }
       const float m_use = (m == -INFINITY) ? 0.f : m;
-      // P = 2^(scale s - m) as bf16 pairs over the first 64 columns of S
-      float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // eight independent sum chains
-      uint32_t pk[kBN / 2];
+      // P = 2^(scale s - m) as bf16 pairs over the first 64 columns of S: keys 0-63 first (P columns
+      // 0-31), released to the P V MMA at once, then keys 64-127. Blocks that no row of the warp
+      // masks may take part of the exponentials on the FMA pipe (exp2_poly_pair); masked entries
+      // always go through ex2, which returns exactly 0 for them.
+      const bool poly_ok = kPolyEighths > 0 && !__any_sync(0xffffffffu, kbase + kBN - 1 > row_limit);
+      const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), nm2 = f2_pack(-m_use, -m_use);
+      uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};  // four packed sum chains
 #pragma unroll
-      for (int c = 0; c < kBN; c += 2) {
-        const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c]), a.scale_log2, -m_use));
-        const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), a.scale_log2, -m_use));
-        rs8[(c >> 1) & 7] += p0 + p1;
-        pk[c / 2] = pack_bf16(p0, p1);
-      }
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < kBN / 2; c += 16) tmem_st16(tS + c, pk + c);
-      // S of block j is complete, hence so is P V of block j - 1: O may be rescaled now, before
-      // P V of block j is released below.
-      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 16) {
-          uint32_t orr[16];
-          tmem_ld16(tO + c0, orr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-          tmem_st16(tO + c0, orr);
+        for (int c = 64 * hf; c < 64 * hf + 64; c += 2) {
+          float x0, x1, p0, p1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2), x0, x1);
+          if (((c >> 1) & 7) < kPolyEighths && poly_ok) {
+            exp2_poly_pair(x0, x1, p0, p1);
+          } else {
+            p0 = fast_exp2(x0);
+            p1 = fast_exp2(x1);
+          }
+          rs2[(c >> 1) & 3] = f2_add(rs2[(c >> 1) & 3], f2_pack(p0, p1));
+          pk[(c - 64 * hf) / 2] = pack_bf16(p0, p1);
         }
+        tmem_st16(tS + 32 * hf, pk);
+        tmem_st16(tS + 32 * hf + 16, pk + 16);
+        // S of block j is complete, hence so is P V of block j - 1: O may be rescaled now, before
+        // the first P V of block j is released.
+        if (hf == 0 && j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 16) {
+            uint32_t orr[16];
+            tmem_ld16(tO + c0, orr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+            tmem_st16(tO + c0, orr);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full + 2 * t + hf);
       }
-      l = l * alpha + (((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7])));
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full + t);
+      float rsum[8];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) f2_unpack(rs2[u], rsum[2 * u], rsum[2 * u + 1]);
+      l = l * alpha + (((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) + ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7])));
     }
     if (ok && n_kv > 0) ok = wait_warp(o_done + t, 0);
     tc_fence_after();

@@ -25,15 +25,16 @@
 // P^T is computed while dK and dQ^T of this tile run; dQ^T goes over the dP^T columns once dK has
 // read dS^T, and the next dP^T waits until the drain has read dQ^T. MMAs execute in issue order,
 // which is what makes each overwrite in TMEM safe. dQ is produced transposed (head dim on the TMEM
-// lanes) so that the drain's reductions are coalesced: a warp adds 32 consecutive head-dim columns
-// of one query row per instruction. For D = 64 the dQ^T MMA still runs with M = 128; the upper 64
+// lanes, query rows on the columns), and the fp32 accumulator interleaves groups of four query
+// rows, [B, Hq, Sq_pad / 4, D, 4], so that a lane adds four consecutive rows of its column with one
+// 16-byte vector reduction and a warp instruction covers 512 contiguous bytes. For D = 64 the dQ^T MMA still runs with M = 128; the upper 64
 // TMEM lanes hold values that are never read.
 // TMEM columns: S^T / P^T [0,128), dP^T / dS^T / dQ^T [128,256), dV [256,256+D), dK [384,384+D).
 //
 // Warp roles (320 threads): warps 0-3 scores (one key row per thread; at the end the dK/dV
 // epilogue), warps 4-7 dQ drain (one TMEM lane = one head-dim column per thread: the whole dQ^T
-// row in one tcgen05.ld, TMEM released at once, then coalesced fp32 reductions into the
-// accumulator, 32 consecutive columns per warp instruction),
+// row in one tcgen05.ld, TMEM released at once, then 4-wide fp32 vector reductions into the
+// interleaved accumulator),
 // warp 8 TMA producer (K, V once; Q and dO tiles through a 2-stage ring), warp 9 TMEM allocator
 // and MMA issuer (one elected lane of a converged warp). Every wait is bounded.
 #include <math.h>
@@ -76,7 +77,8 @@ struct BwdArgs {
   float scale_log2;  // scale * log2(e)
   const float* lse2;   // [B, Hq, Sq_pad] lse * log2(e); +inf where a row sees no key or is padding
   const float* delta;  // [B, Hq, Sq_pad]; 0 on padding rows
-  float* dq_acc;       // [B, Sq_pad, Hq, D] fp32
+  float* dq_acc;       // fp32, [B, Hq, Sq_pad / 4, D, 4]: element (b, q, h, d) at
+                       // (((b Hq + h) Sq_pad / 4 + q / 4) D + d) 4 + q % 4
   uint16_t* dk;
   uint16_t* dv;
   int* status;
@@ -89,8 +91,11 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-__device__ __forceinline__ void red_add_f32(float* p, float x) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(x) : "memory");
+// p[0..3] += x[0..3] (fp32 bit patterns) with one vector reduction; p is 16-byte aligned
+__device__ __forceinline__ void red_add_v4_f32(float* p, const uint32_t* x) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(__uint_as_float(x[0])),
+               "f"(__uint_as_float(x[1])), "f"(__uint_as_float(x[2])), "f"(__uint_as_float(x[3]))
+               : "memory");
 }
 
 template <int D>
@@ -434,8 +439,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ dQ drain (warps 4-7)
-    // Thread e holds TMEM lane e = head-dim column d of dQ^T; for each query row q the warp's 32
-    // lanes add 32 consecutive columns (128 contiguous bytes) into the accumulator.
+    // Thread e holds TMEM lane e = head-dim column d of dQ^T; for each group of four query rows the
+    // warp's 32 lanes add 32 consecutive columns x 4 rows (512 contiguous bytes) into the
+    // interleaved accumulator.
     const int wq = warp - 4;
     const int d = wq * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
@@ -444,7 +450,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool r = mbar_wait(bar, parity, abort, a.status);
       return __all_sync(0xffffffffu, r);
     };
-    const long long row_stride = static_cast<long long>(a.Hq) * D;
     for (int j = 0; j < n_it; ++j) {
       const int h = g * G + j / n_q;
       const int q0 = (qt0 + j % n_q) * kBM;
@@ -459,12 +464,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_free);
       if (d < D) {  // at D = 64 warps 6 and 7 hold no dQ column
-        float* acc = a.dq_acc + ((static_cast<long long>(b) * a.Sq_pad + q0) * a.Hq + h) * D + d;
+        // rows q0 + 4i .. q0 + 4i + 3 of column d: 16 contiguous bytes at acc + 4 D i
+        float* acc = a.dq_acc + ((static_cast<long long>(b) * a.Hq + h) * a.Sq_pad + q0) * D + 4 * d;
 #pragma unroll
-        for (int c = 0; c < kBM; ++c) {  // a running pointer: one 64-bit add per row, no address table
-          red_add_f32(acc, __uint_as_float(r[c]));
-          acc += row_stride;
-        }
+        for (int i = 0; i < kBM / 4; ++i) red_add_v4_f32(acc + 4 * D * i, r + 4 * i);
       }
     }
   }
@@ -506,7 +509,9 @@ __global__ void __launch_bounds__(128) bwd_prep_kernel(const uint16_t* __restric
       s = bf16_lo(x) * bf16_lo(y) + bf16_hi(x) * bf16_hi(y);
     }
   }
-  const long long abase = row * D + lane * DPL;  // padded accumulator row (b, i, h)
+  // zero D accumulator values per row: together the rows cover the whole accumulator, whatever
+  // its internal order
+  const long long abase = row * D + lane * DPL;
   if constexpr (DPL == 4)
     *reinterpret_cast<float4*>(dq_acc + abase) = make_float4(0.f, 0.f, 0.f, 0.f);
   else
@@ -520,25 +525,31 @@ __global__ void __launch_bounds__(128) bwd_prep_kernel(const uint16_t* __restric
   }
 }
 
-// dQ = scale * accumulator -> bf16, eight elements per thread (real rows only).
+// dQ = scale * accumulator -> bf16. A thread takes two adjacent head-dim columns of one group of
+// four query rows (two float4 of the interleaved accumulator) and writes a bf16 pair to each of
+// the four rows that exist.
 __global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const float* __restrict__ acc,
-                                                             uint16_t* __restrict__ dq, long long n8, int Sq,
-                                                             int Sq_pad, int row8, float scale) {
+                                                             uint16_t* __restrict__ dq, int B, int Hq, int Sq,
+                                                             int Sq_pad, int D, float scale) {
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n8) return;
-  // output group i lies in output row r = b * Sq + q (row8 groups per row); the accumulator row of
-  // the same (b, q) is b * Sq_pad + q
-  const long long r = i / row8, off = i % row8;
-  const long long b = r / Sq, q = r % Sq;
-  const float4* src = reinterpret_cast<const float4*>(acc) + ((b * Sq_pad + q) * row8 + off) * 2;
-  const float4 x = src[0];
-  const float4 y = src[1];
-  uint4 w;
-  w.x = pack_bf16(x.x * scale, x.y * scale);
-  w.y = pack_bf16(x.z * scale, x.w * scale);
-  w.z = pack_bf16(y.x * scale, y.y * scale);
-  w.w = pack_bf16(y.z * scale, y.w * scale);
-  reinterpret_cast<uint4*>(dq)[i] = w;
+  const int half_d = D / 2, groups = Sq_pad / 4;
+  if (i >= static_cast<long long>(B) * Hq * groups * half_d) return;
+  const int dp = static_cast<int>(i % half_d);
+  long long t = i / half_d;
+  const int g4 = static_cast<int>(t % groups);
+  t /= groups;
+  const int h = static_cast<int>(t % Hq);
+  const long long b = t / Hq;
+  const float4* src = reinterpret_cast<const float4*>(acc) + ((b * Hq + h) * groups + g4) * D + 2 * dp;
+  const float4 x = src[0];  // column 2 dp, rows 4 g4 .. 4 g4 + 3
+  const float4 y = src[1];  // column 2 dp + 1
+  const float xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int q = 4 * g4 + e;
+    if (q < Sq)
+      *reinterpret_cast<uint32_t*>(dq + ((b * Sq + q) * Hq + h) * D + 2 * dp) = pack_bf16(xs[e] * scale, ys[e] * scale);
+  }
 }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -595,12 +606,11 @@ cudaError_t launch_bwd_sm100_d(const Problem& p, const void* q, const void* k, c
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
-  const int row8 = p.Hq * D / 8;
-  const long long n8 = static_cast<long long>(p.B) * p.Sq * row8;
+  const long long n_conv = static_cast<long long>(p.B) * p.Hq * (Sq_pad / 4) * (D / 2);
   {
     LaunchScope ls("bwd_dq_convert", st);
-    bwd_dq_convert_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, st>>>(
-        dq_acc, static_cast<uint16_t*>(dq), n8, p.Sq, Sq_pad, row8, p.scale);
+    bwd_dq_convert_kernel<<<static_cast<unsigned>((n_conv + 255) / 256), 256, 0, st>>>(
+        dq_acc, static_cast<uint16_t*>(dq), p.B, p.Hq, p.Sq, Sq_pad, D, p.scale);
   }
   return cudaGetLastError();
 }

@@ -73,7 +73,8 @@ struct DecCfg {
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kDecStages * kBlkBytes;
   static constexpr int kOffBar = 2 * kDecStages * kBlkBytes;
-  static constexpr int kSmemBytes = kOffBar + 2 * kDecStages * 8 + 16 + 1024;
+  static constexpr int kOffP = kOffBar + 2 * kDecStages * 8 + 16;  // [4 warps][32 keys][4 heads] (p, p)
+  static constexpr int kSmemBytes = kOffP + 4 * kDecBlk * 4 * 8 + 1024;
 };
 
 __device__ __forceinline__ bool dec_wait_drain(uint64_t* bar, uint32_t parity) {
@@ -108,7 +109,9 @@ __global__ void __launch_bounds__(kDecThreads, 3)
   __shared__ __align__(16) float qs[GT][D];
   __shared__ float red_m[4][GT];
   __shared__ float red_l[4][GT];
-  __shared__ __align__(16) float red_o[4][GT][D];
+  // The four compute warps' unnormalised outputs, merged at the end, reuse the K ring (every block
+  // has been consumed by then).
+  float(*red_o)[GT][D] = reinterpret_cast<float(*)[GT][D]>(sK);
 
   const int c = blockIdx.x, n = blockIdx.z;
   const int G = Hq / Hkv, npass = G / GT;
@@ -182,15 +185,21 @@ __global__ void __launch_bounds__(kDecThreads, 3)
   }
 
   // ------------------------------------------------------------------ compute warps
-  float m[GT], ls[GT], acc[GT][DPL];
+  // Pairs of fp32 values go through the packed f32x2 instructions: the scores accumulate two
+  // head-dim products per instruction, the outputs two value dimensions per instruction.
+  constexpr int PPL = DPL / 2;  // value-dimension pairs per lane
+  float m[GT], ls[GT];
+  uint64_t acc2[GT][PPL];
 #pragma unroll
   for (int t = 0; t < GT; ++t) {
     m[t] = -INFINITY;
     ls[t] = 0.f;
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[t][e] = 0.f;
+    for (int e = 0; e < PPL; ++e) acc2[t][e] = 0ull;
   }
   const int vd = lane * DPL;  // this lane's value dimensions: vd .. vd + DPL - 1
+  // this warp's block probabilities as (p, p) pairs: [32 keys][GT] x 8 bytes
+  uint64_t* sp = reinterpret_cast<uint64_t*>(smem + C::kOffP) + warp * kDecBlk * 4;
   for (int bk = warp; bk < nblk; bk += 4) {
     const int s = bk % kDecStages;
     const bool ok = mbar_wait(full + s, (bk / kDecStages) & 1, abort, status);
@@ -199,69 +208,76 @@ __global__ void __launch_bounds__(kDecThreads, 3)
     const uint8_t* vb = sV + s * C::kBlkBytes;
     const int nk = min(kDecBlk, k1 - (k0 + bk * kDecBlk));
     const bool valid = lane < nk;
-    // scores of this lane's key for the GT heads (base-2 units: q carries scale * log2 e)
-    float sc[GT];
+    // scores of this lane's key for the GT heads (base-2 units: q carries scale * log2 e); two
+    // independent pair accumulators per head
+    uint64_t sc2[GT][2];
 #pragma unroll
-    for (int t = 0; t < GT; ++t) sc[t] = 0.f;
+    for (int t = 0; t < GT; ++t) sc2[t][0] = sc2[t][1] = 0ull;
 #pragma unroll
     for (int cc = 0; cc < D / 8; ++cc) {
       const uint4 w = *reinterpret_cast<const uint4*>(kb + dec_sw<D>(lane, cc * 8));
-      const float k_[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
-                           bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+      const uint64_t kp0 = f2_pack(bf16_lo(w.x), bf16_hi(w.x)), kp1 = f2_pack(bf16_lo(w.y), bf16_hi(w.y));
+      const uint64_t kp2 = f2_pack(bf16_lo(w.z), bf16_hi(w.z)), kp3 = f2_pack(bf16_lo(w.w), bf16_hi(w.w));
 #pragma unroll
       for (int t = 0; t < GT; ++t) {
         const float4 qa = *reinterpret_cast<const float4*>(&qs[t][8 * cc]);
         const float4 qb = *reinterpret_cast<const float4*>(&qs[t][8 * cc + 4]);
-        float x = sc[t];
-        x = fmaf(qa.x, k_[0], x);
-        x = fmaf(qa.y, k_[1], x);
-        x = fmaf(qa.z, k_[2], x);
-        x = fmaf(qa.w, k_[3], x);
-        x = fmaf(qb.x, k_[4], x);
-        x = fmaf(qb.y, k_[5], x);
-        x = fmaf(qb.z, k_[6], x);
-        x = fmaf(qb.w, k_[7], x);
-        sc[t] = x;
+        sc2[t][0] = f2_fma(f2_pack(qa.x, qa.y), kp0, sc2[t][0]);
+        sc2[t][1] = f2_fma(f2_pack(qa.z, qa.w), kp1, sc2[t][1]);
+        sc2[t][0] = f2_fma(f2_pack(qb.x, qb.y), kp2, sc2[t][0]);
+        sc2[t][1] = f2_fma(f2_pack(qb.z, qb.w), kp3, sc2[t][1]);
       }
     }
     float p[GT];
 #pragma unroll
     for (int t = 0; t < GT; ++t) {
-      const float st = valid ? sc[t] : -INFINITY;
+      float a0, a1, b0, b1;
+      f2_unpack(sc2[t][0], a0, a1);
+      f2_unpack(sc2[t][1], b0, b1);
+      const float st = valid ? (a0 + a1) + (b0 + b1) : -INFINITY;
       const float mn = fmaxf(m[t], warp_max(st));  // finite: lane 0's key is valid
       const float alpha = fast_exp2(m[t] - mn);     // 2^(-inf) = 0 on the first block
       p[t] = valid ? fast_exp2(st - mn) : 0.f;
       ls[t] = ls[t] * alpha + p[t];
+      const uint64_t al2 = f2_pack(alpha, alpha);
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) acc[t][e] *= alpha;
+      for (int e = 0; e < PPL; ++e) acc2[t][e] = f2_mul(acc2[t][e], al2);
       m[t] = mn;
     }
+    // this lane's key probabilities, duplicated into pairs, for the whole warp
+#pragma unroll
+    for (int t = 0; t < GT; ++t) sp[lane * 4 + t] = f2_pack(p[t], p[t]);
+    __syncwarp();
     for (int j = 0; j < nk; ++j) {
       const uint8_t* vr = vb + dec_sw<D>(j, vd);
-      float vv[DPL];
+      uint64_t vp[PPL];
       if constexpr (DPL == 4) {
         const uint2 w = *reinterpret_cast<const uint2*>(vr);
-        vv[0] = bf16_lo(w.x);
-        vv[1] = bf16_hi(w.x);
-        vv[2] = bf16_lo(w.y);
-        vv[3] = bf16_hi(w.y);
+        vp[0] = f2_pack(bf16_lo(w.x), bf16_hi(w.x));
+        vp[1] = f2_pack(bf16_lo(w.y), bf16_hi(w.y));
       } else {
         const uint32_t w = *reinterpret_cast<const uint32_t*>(vr);
-        vv[0] = bf16_lo(w);
-        vv[1] = bf16_hi(w);
+        vp[0] = f2_pack(bf16_lo(w), bf16_hi(w));
       }
 #pragma unroll
       for (int t = 0; t < GT; ++t) {
-        const float pj = __shfl_sync(0xffffffffu, p[t], j);
+        const uint64_t pj = sp[j * 4 + t];  // same address in every lane: a broadcast
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) acc[t][e] = fmaf(pj, vv[e], acc[t][e]);
+        for (int e = 0; e < PPL; ++e) acc2[t][e] = f2_fma(pj, vp[e], acc2[t][e]);
       }
     }
-    __syncwarp();
+    __syncwarp();  // sp is rewritten by the next block
     if (lane == 0) mbar_arrive(empty + s);
   }
+  float acc[GT][DPL];
+#pragma unroll
+  for (int t = 0; t < GT; ++t)
+#pragma unroll
+    for (int e = 0; e < PPL; ++e) f2_unpack(acc2[t][e], acc[t][2 * e], acc[t][2 * e + 1]);
 
-  // merge the four warps' triples (a warp that saw no block holds the identity)
+  // merge the four warps' triples (a warp that saw no block holds the identity); red_o overlays the
+  // K ring, so every compute warp must be done reading it first
+  named_barrier(1, 128);
 #pragma unroll
   for (int t = 0; t < GT; ++t) {
     const float lw = warp_sum(ls[t]);

@@ -12,14 +12,14 @@
 // The path is HBM-bound (each K/V byte is read once, about 4 flop per byte), so the split kernel is
 // CUDA-core code built to keep many bytes in flight without spending registers on them. A CTA
 // covers one (chunk, kv head, stream) and all the query heads of that kv head's group, so each K/V
-// row is fetched once for GT query heads. One producer warp streams 32-key K and V blocks of the
-// chunk with TMA tile loads (128-byte swizzle) into a 4-stage shared-memory ring; compute warp w
-// takes blocks w, w+4, ... and keeps its own online-softmax triples for the GT heads: each lane
-// scores one key for all GT heads (its K row read once from shared memory) and owns D/32 value
-// dimensions of every head (each V row read once per lane). The four warps' triples are merged
-// with the monoid at the end.
+// row is fetched once for GT query heads. One producer warp streams 16-key K and V blocks of the
+// chunk with TMA tile loads (128-byte swizzle) into an 8-stage shared-memory ring; compute warp w
+// takes blocks w, w+4, ... (two stages per warp, so one block lands while the other is used) and
+// keeps its own online-softmax triples for the GT heads: two lanes score one key for all GT heads
+// (each over half of the head dim, its K row read once from shared memory) and each lane owns D/32
+// value dimensions of every head. The four warps' triples are merged with the monoid at the end.
 // The host does not know the cache's row count T (it lives on the device as kv_offsets[N]), so the
-// tensor maps carry a nominal row extent and the kernel issues a 32-row box only when the whole box
+// tensor maps carry a nominal row extent and the kernel issues a 16-row box only when the whole box
 // lies below T; the cache's last partial block is fetched in 16-byte pieces with bulk copies. No
 // copy ever touches memory past the caller's K and V buffers.
 #include <math.h>
@@ -56,11 +56,12 @@ __device__ __forceinline__ int stream_splits(const int* num_splits, int n, int L
   return decode_split_rule(L, max_splits);
 }
 
-constexpr int kDecBlk = 32;              // keys per block (one per lane)
-constexpr int kDecStages = 4;
+constexpr int kDecBlk = 16;              // keys per block (two lanes per key while scoring)
+constexpr int kDecStages = 8;
 // Compute warp w consumes blocks w, w + 4, ... and every stage has a single-arrival "empty" barrier,
 // so a stage must always belong to the same warp: the stage count is a multiple of the four compute
 // warps (otherwise two warps would share a stage and a parity wait could match the wrong phase).
+// With eight stages each warp owns two, so its next block is in flight while it computes one.
 static_assert(kDecStages % 4 == 0, "decode ring stages must be a multiple of the compute warps");
 constexpr int kDecThreads = 160;          // four compute warps + one producer warp
 constexpr int kDecMapRows = 0x7fffffff;   // nominal row extent of the K/V tensor maps
@@ -68,13 +69,12 @@ constexpr int kDecMapRows = 0x7fffffff;   // nominal row extent of the K/V tenso
 template <int D>
 struct DecCfg {
   static constexpr int kAtoms = D / 64;
-  static constexpr int kAtomBytes = kDecBlk * 128;       // 32 rows x 128 bytes
+  static constexpr int kAtomBytes = kDecBlk * 128;       // 16 rows x 128 bytes
   static constexpr int kBlkBytes = kAtoms * kAtomBytes;  // 32 key rows x D bf16
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kDecStages * kBlkBytes;
   static constexpr int kOffBar = 2 * kDecStages * kBlkBytes;
-  static constexpr int kOffP = kOffBar + 2 * kDecStages * 8 + 16;  // [4 warps][32 keys][4 heads] (p, p)
-  static constexpr int kSmemBytes = kOffP + 4 * kDecBlk * 4 * 8 + 1024;
+  static constexpr int kSmemBytes = kOffBar + 2 * kDecStages * 8 + 16 + 1024;
 };
 
 __device__ __forceinline__ bool dec_wait_drain(uint64_t* bar, uint32_t parity) {
@@ -98,7 +98,6 @@ __global__ void __launch_bounds__(kDecThreads, 3)
                         const int* __restrict__ num_splits, int max_splits, int Hq, int Hkv, float scale_log2,
                         float* __restrict__ part_o, float* __restrict__ part_ml, int* status) {
   using C = DecCfg<D>;
-  constexpr int DPL = D / 32;  // value dimensions per lane
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem + C::kOffK;
@@ -106,7 +105,6 @@ __global__ void __launch_bounds__(kDecThreads, 3)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* empty = full + kDecStages;
   volatile int* abort = reinterpret_cast<volatile int*>(empty + kDecStages);
-  __shared__ __align__(16) float qs[GT][D];
   __shared__ float red_m[4][GT];
   __shared__ float red_l[4][GT];
   // The four compute warps' unnormalised outputs, merged at the end, reuse the K ring (every block
@@ -135,11 +133,6 @@ __global__ void __launch_bounds__(kDecThreads, 3)
     *abort = 0;
     fence_mbar_init();
   }
-  for (int e = tid; e < GT * D; e += kDecThreads) {
-    const int t = e / D, d = e - t * D;
-    qs[t][d] = __uint_as_float(static_cast<uint32_t>(q[(static_cast<long long>(n) * Hq + h0 + t) * D + d]) << 16) *
-               scale_log2;
-  }
   __syncthreads();
 
   if (warp == 4) {
@@ -153,8 +146,18 @@ __global__ void __launch_bounds__(kDecThreads, 3)
       const bool tile = row0 + kDecBlk <= T;
       const int nrows = tile ? kDecBlk : min(kDecBlk, k1 - (k0 + bk * kDecBlk));
       bool ok = true;
+      if (lane == 0) ok = mbar_wait(empty + s, ((bk / kDecStages) & 1) ^ 1, abort, status);
+      if (!tile && __shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+        // Rows past the cache's end stay out of the copy; the tensor-core products read every row of
+        // the block (weighted by probability 0), so they must hold finite values: zeros.
+        for (int idx = lane; idx < (kDecBlk - nrows) * (D / 8); idx += 32) {
+          const int r = nrows + idx / (D / 8), d = (idx % (D / 8)) * 8;
+          *reinterpret_cast<uint4*>(sK + s * C::kBlkBytes + dec_sw<D>(r, d)) = make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(sV + s * C::kBlkBytes + dec_sw<D>(r, d)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        __syncwarp();
+      }
       if (lane == 0) {
-        ok = mbar_wait(empty + s, ((bk / kDecStages) & 1) ^ 1, abort, status);
         if (ok) {
           mbar_arrive_expect_tx(full + s, 2u * nrows * D * 2);
           if (tile) {
@@ -185,108 +188,101 @@ __global__ void __launch_bounds__(kDecThreads, 3)
   }
 
   // ------------------------------------------------------------------ compute warps
-  // Pairs of fp32 values go through the packed f32x2 instructions: the scores accumulate two
-  // head-dim products per instruction, the outputs two value dimensions per instruction.
-  constexpr int PPL = DPL / 2;  // value-dimension pairs per lane
-  float m[GT], ls[GT];
-  uint64_t acc2[GT][PPL];
+  // Both contractions of a block run as warp-level tensor-core products (m16n8k16): the GT query
+  // heads are the rows (padded to 16 with zeros), so S^T = Q K^T takes K straight from the ring as
+  // its column operand and P V takes the probabilities straight from the score accumulators.
+  // Lane (g, t) = (lane / 4, lane % 4) holds head g: scores of keys 2t, 2t + 1, 8 + 2t, 9 + 2t of
+  // the block and output columns 8 j + 2t, 8 j + 2t + 1 of every 8-column tile j.
+  const int gq = lane >> 2, tq = lane & 3;
+  const bool head = gq < GT;
+  constexpr int KS = D / 16;  // 16-wide steps over the head dim
+  uint32_t qa[KS], qb[KS];    // Q fragments of head gq (zero for padding rows)
+  {
+    const uint16_t* qrow = q + (static_cast<long long>(n) * Hq + h0 + (head ? gq : 0)) * D;
 #pragma unroll
-  for (int t = 0; t < GT; ++t) {
-    m[t] = -INFINITY;
-    ls[t] = 0.f;
-#pragma unroll
-    for (int e = 0; e < PPL; ++e) acc2[t][e] = 0ull;
+    for (int ks = 0; ks < KS; ++ks) {
+      qa[ks] = head ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq) : 0u;
+      qb[ks] = head ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * tq) : 0u;
+    }
   }
-  const int vd = lane * DPL;  // this lane's value dimensions: vd .. vd + DPL - 1
-  // this warp's block probabilities as (p, p) pairs: [32 keys][GT] x 8 bytes
-  uint64_t* sp = reinterpret_cast<uint64_t*>(smem + C::kOffP) + warp * kDecBlk * 4;
+  float o[D / 8][4];
+#pragma unroll
+  for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float mrow = -INFINITY, lrow = 0.f;  // head gq: running max (base 2) and this lane's share of the sum
+  // ldmatrix row owned by this lane: matrix mi = lane / 8, row ri = lane % 8
+  const int mi = lane >> 3, ri = lane & 7;
   for (int bk = warp; bk < nblk; bk += 4) {
     const int s = bk % kDecStages;
     const bool ok = mbar_wait(full + s, (bk / kDecStages) & 1, abort, status);
     if (!__all_sync(0xffffffffu, ok)) break;
-    const uint8_t* kb = sK + s * C::kBlkBytes;
-    const uint8_t* vb = sV + s * C::kBlkBytes;
+    const uint32_t kb = smem_u32(sK + s * C::kBlkBytes);
+    const uint32_t vb = smem_u32(sV + s * C::kBlkBytes);
     const int nk = min(kDecBlk, k1 - (k0 + bk * kDecBlk));
-    const bool valid = lane < nk;
-    // scores of this lane's key for the GT heads (base-2 units: q carries scale * log2 e); two
-    // independent pair accumulators per head
-    uint64_t sc2[GT][2];
+    // S^T for keys 0-7 (s0) and 8-15 (s1)
+    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int t = 0; t < GT; ++t) sc2[t][0] = sc2[t][1] = 0ull;
+    for (int ks = 0; ks < KS; ++ks) {
+      uint32_t b00, b01, b10, b11;  // matrices: keys 8 (mi / 2) + ri, head dims 16 ks + 8 (mi % 2) ..
+      ldsm_x4(kb + dec_sw<D>(ri + 8 * (mi >> 1), 16 * ks + 8 * (mi & 1)), b00, b01, b10, b11);
+      mma_16816(s0, qa[ks], 0u, qb[ks], 0u, b00, b01);
+      mma_16816(s1, qa[ks], 0u, qb[ks], 0u, b10, b11);
+    }
+    float x[4] = {s0[0], s0[1], s1[0], s1[1]};
+    const int kx[4] = {2 * tq, 2 * tq + 1, 8 + 2 * tq, 9 + 2 * tq};
+    float bm = -INFINITY;
 #pragma unroll
-    for (int cc = 0; cc < D / 8; ++cc) {
-      const uint4 w = *reinterpret_cast<const uint4*>(kb + dec_sw<D>(lane, cc * 8));
-      const uint64_t kp0 = f2_pack(bf16_lo(w.x), bf16_hi(w.x)), kp1 = f2_pack(bf16_lo(w.y), bf16_hi(w.y));
-      const uint64_t kp2 = f2_pack(bf16_lo(w.z), bf16_hi(w.z)), kp3 = f2_pack(bf16_lo(w.w), bf16_hi(w.w));
+    for (int e = 0; e < 4; ++e) {
+      x[e] = kx[e] < nk ? x[e] * scale_log2 : -INFINITY;
+      bm = fmaxf(bm, x[e]);
+    }
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));  // block max of head gq (key 0 is valid)
+    // lazy rescale: the reference max moves only when the block max exceeds it by more than 8
+    float alpha = 1.f;
+    if (bm > mrow + 8.f || mrow == -INFINITY) {
+      alpha = (mrow == -INFINITY) ? 0.f : fast_exp2(mrow - bm);
+      mrow = bm;
+    }
+    if (__any_sync(0xffffffffu, alpha != 1.f)) {
+      lrow *= alpha;
 #pragma unroll
-      for (int t = 0; t < GT; ++t) {
-        const float4 qa = *reinterpret_cast<const float4*>(&qs[t][8 * cc]);
-        const float4 qb = *reinterpret_cast<const float4*>(&qs[t][8 * cc + 4]);
-        sc2[t][0] = f2_fma(f2_pack(qa.x, qa.y), kp0, sc2[t][0]);
-        sc2[t][1] = f2_fma(f2_pack(qa.z, qa.w), kp1, sc2[t][1]);
-        sc2[t][0] = f2_fma(f2_pack(qb.x, qb.y), kp2, sc2[t][0]);
-        sc2[t][1] = f2_fma(f2_pack(qb.z, qb.w), kp3, sc2[t][1]);
+      for (int j = 0; j < D / 8; ++j) {
+        o[j][0] *= alpha;
+        o[j][1] *= alpha;
       }
     }
-    float p[GT];
+    float p[4];
 #pragma unroll
-    for (int t = 0; t < GT; ++t) {
-      float a0, a1, b0, b1;
-      f2_unpack(sc2[t][0], a0, a1);
-      f2_unpack(sc2[t][1], b0, b1);
-      const float st = valid ? (a0 + a1) + (b0 + b1) : -INFINITY;
-      const float mn = fmaxf(m[t], warp_max(st));  // finite: lane 0's key is valid
-      const float alpha = fast_exp2(m[t] - mn);     // 2^(-inf) = 0 on the first block
-      p[t] = valid ? fast_exp2(st - mn) : 0.f;
-      ls[t] = ls[t] * alpha + p[t];
-      const uint64_t al2 = f2_pack(alpha, alpha);
-#pragma unroll
-      for (int e = 0; e < PPL; ++e) acc2[t][e] = f2_mul(acc2[t][e], al2);
-      m[t] = mn;
+    for (int e = 0; e < 4; ++e) {
+      p[e] = head ? fast_exp2(x[e] - mrow) : 0.f;  // 2^(-inf) = 0 for keys past the block's end
+      lrow += p[e];
     }
-    // this lane's key probabilities, duplicated into pairs, for the whole warp
+    const uint32_t pa0 = pack_bf16(p[0], p[1]), pa2 = pack_bf16(p[2], p[3]);
+    // O += P V over pairs of 8-column tiles
 #pragma unroll
-    for (int t = 0; t < GT; ++t) sp[lane * 4 + t] = f2_pack(p[t], p[t]);
+    for (int jp = 0; jp < D / 16; ++jp) {
+      uint32_t v0, v1, v2, v3;  // matrices: keys 8 (mi % 2) + ri, head dims 16 jp + 8 (mi / 2) ..
+      ldsm_x4_trans(vb + dec_sw<D>(ri + 8 * (mi & 1), 16 * jp + 8 * (mi >> 1)), v0, v1, v2, v3);
+      mma_16816(o[2 * jp], pa0, 0u, pa2, 0u, v0, v1);
+      mma_16816(o[2 * jp + 1], pa0, 0u, pa2, 0u, v2, v3);
+    }
     __syncwarp();
-    for (int j = 0; j < nk; ++j) {
-      const uint8_t* vr = vb + dec_sw<D>(j, vd);
-      uint64_t vp[PPL];
-      if constexpr (DPL == 4) {
-        const uint2 w = *reinterpret_cast<const uint2*>(vr);
-        vp[0] = f2_pack(bf16_lo(w.x), bf16_hi(w.x));
-        vp[1] = f2_pack(bf16_lo(w.y), bf16_hi(w.y));
-      } else {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(vr);
-        vp[0] = f2_pack(bf16_lo(w), bf16_hi(w));
-      }
-#pragma unroll
-      for (int t = 0; t < GT; ++t) {
-        const uint64_t pj = sp[j * 4 + t];  // same address in every lane: a broadcast
-#pragma unroll
-        for (int e = 0; e < PPL; ++e) acc2[t][e] = f2_fma(pj, vp[e], acc2[t][e]);
-      }
-    }
-    __syncwarp();  // sp is rewritten by the next block
     if (lane == 0) mbar_arrive(empty + s);
   }
-  float acc[GT][DPL];
-#pragma unroll
-  for (int t = 0; t < GT; ++t)
-#pragma unroll
-    for (int e = 0; e < PPL; ++e) f2_unpack(acc2[t][e], acc[t][2 * e], acc[t][2 * e + 1]);
+  lrow += __shfl_xor_sync(0xffffffffu, lrow, 1);
+  lrow += __shfl_xor_sync(0xffffffffu, lrow, 2);
 
   // merge the four warps' triples (a warp that saw no block holds the identity); red_o overlays the
   // K ring, so every compute warp must be done reading it first
   named_barrier(1, 128);
-#pragma unroll
-  for (int t = 0; t < GT; ++t) {
-    const float lw = warp_sum(ls[t]);
-    if (lane == 0) {
-      red_m[warp][t] = m[t];
-      red_l[warp][t] = lw;
+  if (head) {
+    if (tq == 0) {
+      red_m[warp][gq] = mrow;
+      red_l[warp][gq] = lrow;
     }
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) red_o[warp][t][vd + e] = acc[t][e];
+    for (int j = 0; j < D / 8; ++j)
+      *reinterpret_cast<float2*>(&red_o[warp][gq][8 * j + 2 * tq]) = make_float2(o[j][0], o[j][1]);
   }
   named_barrier(1, 128);  // the four compute warps only
   for (int e = tid; e < GT * D; e += 128) {

@@ -263,6 +263,11 @@ __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// Arrives at a named barrier without waiting (the waiting side uses named_barrier).
+__device__ __forceinline__ void named_barrier_arrive(int id, int threads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // Orders this thread's generic-proxy shared-memory writes before later async-proxy reads
 // (tensor-core operand fetch, TMA store).
 __device__ __forceinline__ void fence_proxy_async_smem() {

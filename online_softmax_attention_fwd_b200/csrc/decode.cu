@@ -9,20 +9,24 @@
 // identity (-inf, 0, 0), a weight 2^(-inf - M) taken as 0. The merge is the same one the split
 // kernel uses between its four warps, so the result does not depend on how the keys were cut.
 //
-// The path is HBM-bound (each K/V byte is read once, about 4 flop per byte), so the split kernel is
-// CUDA-core code built to keep many bytes in flight without spending registers on them. A CTA
-// covers one (chunk, kv head, stream) and all the query heads of that kv head's group, so each K/V
-// row is fetched once for GT query heads. One producer warp streams 16-key K and V blocks of the
-// chunk with TMA tile loads (128-byte swizzle) into an 8-stage shared-memory ring; compute warp w
-// takes blocks w, w+4, ... (two stages per warp, so one block lands while the other is used) and
-// keeps its own online-softmax triples for the GT heads: two lanes score one key for all GT heads
-// (each over half of the head dim, its K row read once from shared memory) and each lane owns D/32
-// value dimensions of every head. The four warps' triples are merged with the monoid at the end.
+// The path is HBM-bound (each K/V byte is read once, about 4 flop per byte). The split kernel is a
+// persistent grid (three CTAs per SM) that walks a static list of work items, one item per
+// (chunk, kv head, stream) covering all GT query heads of that kv head's group, so each K/V row is
+// fetched once for GT query heads. One producer warp streams the items' 16-key K and V blocks with
+// TMA tile loads (128-byte swizzle) into an 8-stage shared-memory ring, without a pause between
+// items, and fetches each item's query rows with a bulk copy; compute warp w takes the ring's
+// blocks w, w+4, ... (two stages per warp, so one block lands while the other is used). Both
+// contractions of a block are warp-level tensor-core products: the GT heads are too few rows for
+// tcgen05 (M >= 64) and would waste 16x there, against 4x in m16n8k16. At the end of an item
+// warps 1-3 leave their triples in shared memory and warp 0 merges them with its own and writes
+// the item's partial triple.
 // The host does not know the cache's row count T (it lives on the device as kv_offsets[N]), so the
 // tensor maps carry a nominal row extent and the kernel issues a 16-row box only when the whole box
 // lies below T; the cache's last partial block is fetched in 16-byte pieces with bulk copies. No
 // copy ever touches memory past the caller's K and V buffers.
 #include <math.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -64,18 +68,55 @@ constexpr int kDecStages = 8;
 // With eight stages each warp owns two, so its next block is in flight while it computes one.
 static_assert(kDecStages % 4 == 0, "decode ring stages must be a multiple of the compute warps");
 constexpr int kDecThreads = 160;          // four compute warps + one producer warp
+constexpr int kDecCtasPerSm = 3;
 constexpr int kDecMapRows = 0x7fffffff;   // nominal row extent of the K/V tensor maps
 
 template <int D>
 struct DecCfg {
   static constexpr int kAtoms = D / 64;
   static constexpr int kAtomBytes = kDecBlk * 128;       // 16 rows x 128 bytes
-  static constexpr int kBlkBytes = kAtoms * kAtomBytes;  // 32 key rows x D bf16
+  static constexpr int kBlkBytes = kAtoms * kAtomBytes;  // 16 key rows x D bf16
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kDecStages * kBlkBytes;
-  static constexpr int kOffBar = 2 * kDecStages * kBlkBytes;
-  static constexpr int kSmemBytes = kOffBar + 2 * kDecStages * 8 + 16 + 1024;
+  static constexpr int kOffQ = 2 * kDecStages * kBlkBytes;  // [2 items][<= 4 heads][D] bf16
+  static constexpr int kQBuf = 4 * D * 2;
+  static constexpr int kOffDep = kOffQ + 2 * kQBuf;         // warps 1-3: [3][<= 4 heads][D] fp32
+  static constexpr int kOffBar = kOffDep + 3 * 4 * D * 4;
+  static constexpr int kNumBars = 2 * kDecStages + 4;       // full, empty, q_full[2], q_empty[2]
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;   // abort flag, then the deposits' (m, l)
+  static constexpr int kSmemBytes = kOffMisc + 16 + 2 * 3 * 4 * 4 + 1024;
 };
+
+// One work item: the key chunk c of stream n for the query heads h0 .. h0 + GT - 1 of kv head g.
+struct DecItem {
+  int n, c, g, h0, start, k0, k1, nblk;
+};
+
+// Item slot idx -> item; false for slots past the stream's split count. Slots are ordered chunk
+// index slowest, so the first chunks of every stream and kv head come first.
+template <int GT>
+__device__ __forceinline__ bool dec_item(long long idx, int N, int Hq, int Hkv, const int* offsets,
+                                         const int* num_splits, int max_splits, DecItem& it) {
+  const int G = Hq / Hkv, npass = G / GT, NG = Hkv * npass;
+  const long long per_c = static_cast<long long>(N) * NG;
+  const int c = static_cast<int>(idx / per_c);
+  const int r = static_cast<int>(idx - c * per_c);
+  const int n = r / NG, gi = r - (r / NG) * NG;
+  const int start = offsets[n];
+  const int L = offsets[n + 1] - start;
+  const int C_n = stream_splits(num_splits, n, L, max_splits);
+  if (c >= C_n) return false;
+  const int chunk = (L + C_n - 1) / C_n;
+  it.n = n;
+  it.c = c;
+  it.g = gi / npass;
+  it.h0 = it.g * G + (gi % npass) * GT;
+  it.start = start;
+  it.k0 = min(L, c * chunk);
+  it.k1 = min(L, it.k0 + chunk);
+  it.nblk = (it.k1 - it.k0 + kDecBlk - 1) / kDecBlk;
+  return true;
+}
 
 __device__ __forceinline__ bool dec_wait_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
@@ -91,7 +132,7 @@ __device__ __forceinline__ uint32_t dec_sw(int r, int d) {
 }
 
 template <int D, int GT>
-__global__ void __launch_bounds__(kDecThreads, 3)
+__global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
                         const uint16_t* __restrict__ v, const int* __restrict__ offsets, int N,
@@ -102,33 +143,27 @@ __global__ void __launch_bounds__(kDecThreads, 3)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem + C::kOffK;
   uint8_t* sV = smem + C::kOffV;
+  uint8_t* sQ = smem + C::kOffQ;
+  float* dep = reinterpret_cast<float*>(smem + C::kOffDep);  // [3][GT][D]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* empty = full + kDecStages;
-  volatile int* abort = reinterpret_cast<volatile int*>(empty + kDecStages);
-  __shared__ float red_m[4][GT];
-  __shared__ float red_l[4][GT];
-  // The four compute warps' unnormalised outputs, merged at the end, reuse the K ring (every block
-  // has been consumed by then).
-  float(*red_o)[GT][D] = reinterpret_cast<float(*)[GT][D]>(sK);
+  uint64_t* q_full = empty + kDecStages;  // [2]
+  uint64_t* q_empty = q_full + 2;         // [2]
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc);
+  float* dep_m = reinterpret_cast<float*>(smem + C::kOffMisc + 16);  // [3][4]
+  float* dep_l = dep_m + 12;                                         // [3][4]
 
-  const int c = blockIdx.x, n = blockIdx.z;
   const int G = Hq / Hkv, npass = G / GT;
-  const int g = blockIdx.y / npass;
-  const int h0 = g * G + (blockIdx.y % npass) * GT;
-  const int start = offsets[n];
-  const int L = offsets[n + 1] - start;
-  const int C_n = stream_splits(num_splits, n, L, max_splits);
-  if (c >= C_n) return;  // uniform over the CTA; the combine reads only the first C_n slots
-  const int chunk = (L + C_n - 1) / C_n;
-  const int k0 = min(L, c * chunk);
-  const int k1 = min(L, k0 + chunk);
-  const int nblk = (k1 - k0 + kDecBlk - 1) / kDecBlk;
-
+  const long long n_slots = static_cast<long long>(N) * Hkv * npass * max_splits;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < kDecStages; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);  // each block is consumed by exactly one compute warp
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(q_full + b, 1);
+      mbar_init(q_empty + b, 4);  // every compute warp has read its query fragments
     }
     *abort = 0;
     fence_mbar_init();
@@ -139,174 +174,219 @@ __global__ void __launch_bounds__(kDecThreads, 3)
     // ---------------------------------------------------------------- producer
     const int T = min(offsets[N], kDecMapRows);  // no box may reach past the cache
     const long long rs = static_cast<long long>(Hkv) * D;
-    int issued = 0;
-    for (int bk = 0; bk < nblk; ++bk) {
-      const int s = bk % kDecStages;
-      const int row0 = start + k0 + bk * kDecBlk;
-      const bool tile = row0 + kDecBlk <= T;
-      const int nrows = tile ? kDecBlk : min(kDecBlk, k1 - (k0 + bk * kDecBlk));
-      bool ok = true;
-      if (lane == 0) ok = mbar_wait(empty + s, ((bk / kDecStages) & 1) ^ 1, abort, status);
-      if (!tile && __shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
-        // Rows past the cache's end stay out of the copy; the tensor-core products read every row of
-        // the block (weighted by probability 0), so they must hold finite values: zeros.
-        for (int idx = lane; idx < (kDecBlk - nrows) * (D / 8); idx += 32) {
-          const int r = nrows + idx / (D / 8), d = (idx % (D / 8)) * 8;
-          *reinterpret_cast<uint4*>(sK + s * C::kBlkBytes + dec_sw<D>(r, d)) = make_uint4(0u, 0u, 0u, 0u);
-          *reinterpret_cast<uint4*>(sV + s * C::kBlkBytes + dec_sw<D>(r, d)) = make_uint4(0u, 0u, 0u, 0u);
-        }
-        __syncwarp();
-      }
-      if (lane == 0) {
+    long long gb = 0;  // ring position: blocks issued so far
+    int qi = 0;        // items started so far
+    bool ok = true;
+    for (long long idx = blockIdx.x; ok && idx < n_slots; idx += gridDim.x) {
+      DecItem it;
+      if (!dec_item<GT>(idx, N, Hq, Hkv, offsets, num_splits, max_splits, it)) continue;
+      if (lane == 0) {  // the item's GT query rows (contiguous) into query buffer qi % 2
+        ok = mbar_wait(q_empty + (qi & 1), ((qi >> 1) & 1) ^ 1, abort, status);
         if (ok) {
+          mbar_arrive_expect_tx(q_full + (qi & 1), GT * D * 2);
+          bulk_load(sQ + (qi & 1) * C::kQBuf, q + (static_cast<long long>(it.n) * Hq + it.h0) * D, GT * D * 2,
+                    q_full + (qi & 1));
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      ++qi;
+      for (int bk = 0; bk < it.nblk; ++bk) {
+        const int s = static_cast<int>(gb % kDecStages);
+        const int row0 = it.start + it.k0 + bk * kDecBlk;
+        const bool tile = row0 + kDecBlk <= T;
+        const int nrows = tile ? kDecBlk : min(kDecBlk, it.k1 - (it.k0 + bk * kDecBlk));
+        if (lane == 0) ok = mbar_wait(empty + s, static_cast<uint32_t>((gb / kDecStages) & 1) ^ 1, abort, status);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        if (!tile) {
+          // Rows past the cache's end stay out of the copy; the tensor-core products read every row
+          // of the block (weighted by probability 0), so they must hold finite values: zeros.
+          for (int idx2 = lane; idx2 < (kDecBlk - nrows) * (D / 8); idx2 += 32) {
+            const int r = nrows + idx2 / (D / 8), d = (idx2 % (D / 8)) * 8;
+            *reinterpret_cast<uint4*>(sK + s * C::kBlkBytes + dec_sw<D>(r, d)) = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(sV + s * C::kBlkBytes + dec_sw<D>(r, d)) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          __syncwarp();
+        }
+        if (lane == 0) {
           mbar_arrive_expect_tx(full + s, 2u * nrows * D * 2);
           if (tile) {
 #pragma unroll
             for (int at = 0; at < C::kAtoms; ++at) {
-              tma_load_3d(sK + s * C::kBlkBytes + at * C::kAtomBytes, &tmK, full + s, at * 64, g, row0);
-              tma_load_3d(sV + s * C::kBlkBytes + at * C::kAtomBytes, &tmV, full + s, at * 64, g, row0);
+              tma_load_3d(sK + s * C::kBlkBytes + at * C::kAtomBytes, &tmK, full + s, at * 64, it.g, row0);
+              tma_load_3d(sV + s * C::kBlkBytes + at * C::kAtomBytes, &tmV, full + s, at * 64, it.g, row0);
             }
           }
         }
-      }
-      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
-      if (!tile) {
-        // the cache's last rows: 16-byte pieces into the same swizzled places a tile load uses
-        for (int idx = lane; idx < nrows * (D / 8); idx += 32) {
-          const int r = idx / (D / 8), d = (idx % (D / 8)) * 8;
-          bulk_load(sK + s * C::kBlkBytes + dec_sw<D>(r, d), k + (row0 + r) * rs + g * D + d, 16, full + s);
-          bulk_load(sV + s * C::kBlkBytes + dec_sw<D>(r, d), v + (row0 + r) * rs + g * D + d, 16, full + s);
+        __syncwarp();
+        if (!tile) {
+          // the cache's last rows: 16-byte pieces into the same swizzled places a tile load uses
+          for (int idx2 = lane; idx2 < nrows * (D / 8); idx2 += 32) {
+            const int r = idx2 / (D / 8), d = (idx2 % (D / 8)) * 8;
+            bulk_load(sK + s * C::kBlkBytes + dec_sw<D>(r, d), k + (row0 + r) * rs + it.g * D + d, 16, full + s);
+            bulk_load(sV + s * C::kBlkBytes + dec_sw<D>(r, d), v + (row0 + r) * rs + it.g * D + d, 16, full + s);
+          }
         }
+        ++gb;
       }
-      issued = bk + 1;
     }
     // let this CTA's copies land before it can exit (at once on the normal path)
-    if (lane == 0)
-      for (int bk = max(0, issued - kDecStages); bk < issued; ++bk)
-        dec_wait_drain(full + bk % kDecStages, (bk / kDecStages) & 1);
+    if (lane == 0) {
+      for (long long b = max(0ll, gb - kDecStages); b < gb; ++b)
+        dec_wait_drain(full + b % kDecStages, static_cast<uint32_t>((b / kDecStages) & 1));
+      for (int i = max(0, qi - 2); i < qi; ++i) dec_wait_drain(q_full + (i & 1), (i >> 1) & 1);
+    }
     return;
   }
 
   // ------------------------------------------------------------------ compute warps
-  // Both contractions of a block run as warp-level tensor-core products (m16n8k16): the GT query
-  // heads are the rows (padded to 16 with zeros), so S^T = Q K^T takes K straight from the ring as
-  // its column operand and P V takes the probabilities straight from the score accumulators.
   // Lane (g, t) = (lane / 4, lane % 4) holds head g: scores of keys 2t, 2t + 1, 8 + 2t, 9 + 2t of
-  // the block and output columns 8 j + 2t, 8 j + 2t + 1 of every 8-column tile j.
+  // a block and output columns 8 j + 2t, 8 j + 2t + 1 of every 8-column tile j. The GT heads are
+  // the rows of the m16n8k16 products (padded to 16 with zeros), so S^T = Q K^T takes K straight
+  // from the ring as its column operand and P V takes the probabilities straight from the score
+  // accumulators.
   const int gq = lane >> 2, tq = lane & 3;
   const bool head = gq < GT;
   constexpr int KS = D / 16;  // 16-wide steps over the head dim
-  uint32_t qa[KS], qb[KS];    // Q fragments of head gq (zero for padding rows)
-  {
-    const uint16_t* qrow = q + (static_cast<long long>(n) * Hq + h0 + (head ? gq : 0)) * D;
+  const int mi = lane >> 3, ri = lane & 7;  // ldmatrix: this lane addresses row ri of matrix mi
+  long long gb = 0;  // ring position of the current item's first block
+  int qi = 0;
+  bool ok = true;    // false once a wait has failed: the warp then only keeps the barrier protocol
+  for (long long idx = blockIdx.x; idx < n_slots; idx += gridDim.x) {
+    DecItem it;
+    if (!dec_item<GT>(idx, N, Hq, Hkv, offsets, num_splits, max_splits, it)) continue;
+    // this item's query rows (bf16) in shared memory; each block reads its Q fragments from there
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(q_full + (qi & 1), (qi >> 1) & 1, abort, status)) != 0;
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(sQ + (qi & 1) * C::kQBuf) + (head ? gq : 0) * (D / 2);
+    const int qbuf = qi & 1;
+    ++qi;
+    float o[D / 8][4];
 #pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      qa[ks] = head ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq) : 0u;
-      qb[ks] = head ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * tq) : 0u;
-    }
-  }
-  float o[D / 8][4];
+    for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    float mrow = -INFINITY, lrow = 0.f;  // head gq: running max (base 2) and this lane's share of the sum
+    for (int bk = (warp - static_cast<int>(gb & 3)) & 3; ok && bk < it.nblk; bk += 4) {
+      const long long gbk = gb + bk;
+      const int s = static_cast<int>(gbk % kDecStages);
+      ok = __all_sync(0xffffffffu, mbar_wait(full + s, static_cast<uint32_t>((gbk / kDecStages) & 1), abort,
+                                             status)) != 0;
+      if (!ok) break;
+      const uint32_t kb = smem_u32(sK + s * C::kBlkBytes);
+      const uint32_t vb = smem_u32(sV + s * C::kBlkBytes);
+      const int nk = min(kDecBlk, it.k1 - (it.k0 + bk * kDecBlk));
+      // S^T for keys 0-7 (s0) and 8-15 (s1)
+      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-  float mrow = -INFINITY, lrow = 0.f;  // head gq: running max (base 2) and this lane's share of the sum
-  // ldmatrix row owned by this lane: matrix mi = lane / 8, row ri = lane % 8
-  const int mi = lane >> 3, ri = lane & 7;
-  for (int bk = warp; bk < nblk; bk += 4) {
-    const int s = bk % kDecStages;
-    const bool ok = mbar_wait(full + s, (bk / kDecStages) & 1, abort, status);
-    if (!__all_sync(0xffffffffu, ok)) break;
-    const uint32_t kb = smem_u32(sK + s * C::kBlkBytes);
-    const uint32_t vb = smem_u32(sV + s * C::kBlkBytes);
-    const int nk = min(kDecBlk, k1 - (k0 + bk * kDecBlk));
-    // S^T for keys 0-7 (s0) and 8-15 (s1)
-    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      uint32_t b00, b01, b10, b11;  // matrices: keys 8 (mi / 2) + ri, head dims 16 ks + 8 (mi % 2) ..
-      ldsm_x4(kb + dec_sw<D>(ri + 8 * (mi >> 1), 16 * ks + 8 * (mi & 1)), b00, b01, b10, b11);
-      mma_16816(s0, qa[ks], 0u, qb[ks], 0u, b00, b01);
-      mma_16816(s1, qa[ks], 0u, qb[ks], 0u, b10, b11);
-    }
-    float x[4] = {s0[0], s0[1], s1[0], s1[1]};
-    const int kx[4] = {2 * tq, 2 * tq + 1, 8 + 2 * tq, 9 + 2 * tq};
-    float bm = -INFINITY;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      x[e] = kx[e] < nk ? x[e] * scale_log2 : -INFINITY;
-      bm = fmaxf(bm, x[e]);
-    }
-    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));  // block max of head gq (key 0 is valid)
-    // lazy rescale: the reference max moves only when the block max exceeds it by more than 8
-    float alpha = 1.f;
-    if (bm > mrow + 8.f || mrow == -INFINITY) {
-      alpha = (mrow == -INFINITY) ? 0.f : fast_exp2(mrow - bm);
-      mrow = bm;
-    }
-    if (__any_sync(0xffffffffu, alpha != 1.f)) {
-      lrow *= alpha;
-#pragma unroll
-      for (int j = 0; j < D / 8; ++j) {
-        o[j][0] *= alpha;
-        o[j][1] *= alpha;
+      for (int ks = 0; ks < KS; ++ks) {
+        // Q fragments of head gq (zero for the padding rows): head dims 16 ks + 2t .. and + 8
+        const uint32_t qa = head ? qrow[8 * ks + tq] : 0u, qb = head ? qrow[8 * ks + 4 + tq] : 0u;
+        uint32_t b00, b01, b10, b11;  // matrices: keys 8 (mi / 2) + ri, head dims 16 ks + 8 (mi % 2) ..
+        ldsm_x4(kb + dec_sw<D>(ri + 8 * (mi >> 1), 16 * ks + 8 * (mi & 1)), b00, b01, b10, b11);
+        mma_16816(s0, qa, 0u, qb, 0u, b00, b01);
+        mma_16816(s1, qa, 0u, qb, 0u, b10, b11);
       }
-    }
-    float p[4];
+      float x[4] = {s0[0], s0[1], s1[0], s1[1]};
+      const int kx[4] = {2 * tq, 2 * tq + 1, 8 + 2 * tq, 9 + 2 * tq};
+      float bm = -INFINITY;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      p[e] = head ? fast_exp2(x[e] - mrow) : 0.f;  // 2^(-inf) = 0 for keys past the block's end
-      lrow += p[e];
-    }
-    const uint32_t pa0 = pack_bf16(p[0], p[1]), pa2 = pack_bf16(p[2], p[3]);
-    // O += P V over pairs of 8-column tiles
+      for (int e = 0; e < 4; ++e) {
+        x[e] = kx[e] < nk ? x[e] * scale_log2 : -INFINITY;
+        bm = fmaxf(bm, x[e]);
+      }
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));  // block max of head gq (key 0 is valid)
+      // lazy rescale: the reference max moves only when the block max exceeds it by more than 8
+      float alpha = 1.f;
+      if (bm > mrow + 8.f || mrow == -INFINITY) {
+        alpha = (mrow == -INFINITY) ? 0.f : fast_exp2(mrow - bm);
+        mrow = bm;
+      }
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        lrow *= alpha;
 #pragma unroll
-    for (int jp = 0; jp < D / 16; ++jp) {
-      uint32_t v0, v1, v2, v3;  // matrices: keys 8 (mi % 2) + ri, head dims 16 jp + 8 (mi / 2) ..
-      ldsm_x4_trans(vb + dec_sw<D>(ri + 8 * (mi & 1), 16 * jp + 8 * (mi >> 1)), v0, v1, v2, v3);
-      mma_16816(o[2 * jp], pa0, 0u, pa2, 0u, v0, v1);
-      mma_16816(o[2 * jp + 1], pa0, 0u, pa2, 0u, v2, v3);
+        for (int j = 0; j < D / 8; ++j) {
+          o[j][0] *= alpha;
+          o[j][1] *= alpha;
+        }
+      }
+      float p[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        p[e] = head ? fast_exp2(x[e] - mrow) : 0.f;  // 2^(-inf) = 0 for keys past the block's end
+        lrow += p[e];
+      }
+      const uint32_t pa0 = pack_bf16(p[0], p[1]), pa2 = pack_bf16(p[2], p[3]);
+      // O += P V over pairs of 8-column tiles
+#pragma unroll
+      for (int jp = 0; jp < D / 16; ++jp) {
+        uint32_t v0, v1, v2, v3;  // matrices: keys 8 (mi % 2) + ri, head dims 16 jp + 8 (mi / 2) ..
+        ldsm_x4_trans(vb + dec_sw<D>(ri + 8 * (mi & 1), 16 * jp + 8 * (mi >> 1)), v0, v1, v2, v3);
+        mma_16816(o[2 * jp], pa0, 0u, pa2, 0u, v0, v1);
+        mma_16816(o[2 * jp + 1], pa0, 0u, pa2, 0u, v2, v3);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty + s);
     }
+    gb += it.nblk;
     __syncwarp();
-    if (lane == 0) mbar_arrive(empty + s);
-  }
-  lrow += __shfl_xor_sync(0xffffffffu, lrow, 1);
-  lrow += __shfl_xor_sync(0xffffffffu, lrow, 2);
-
-  // merge the four warps' triples (a warp that saw no block holds the identity); red_o overlays the
-  // K ring, so every compute warp must be done reading it first
-  named_barrier(1, 128);
-  if (head) {
-    if (tq == 0) {
-      red_m[warp][gq] = mrow;
-      red_l[warp][gq] = lrow;
-    }
+    if (ok && lane == 0) mbar_arrive(q_empty + qbuf);  // done with this item's query rows
+    lrow += __shfl_xor_sync(0xffffffffu, lrow, 1);
+    lrow += __shfl_xor_sync(0xffffffffu, lrow, 2);
+    // Merge the four warps' triples (a warp that saw no block of the item holds the identity).
+    // Named barrier 1: warps 1-3 have deposited; barrier 2: warp 0 has read the deposits, so they
+    // may be overwritten. Every compute warp passes both for every item, also after a failed wait.
+    if (warp > 0) {
+      if (qi > 1) named_barrier(2, 128);
+      if (head) {
+        float* dw = dep + ((warp - 1) * GT + gq) * D;
+        if (tq == 0) {
+          dep_m[(warp - 1) * 4 + gq] = mrow;
+          dep_l[(warp - 1) * 4 + gq] = lrow;
+        }
 #pragma unroll
-    for (int j = 0; j < D / 8; ++j)
-      *reinterpret_cast<float2*>(&red_o[warp][gq][8 * j + 2 * tq]) = make_float2(o[j][0], o[j][1]);
-  }
-  named_barrier(1, 128);  // the four compute warps only
-  for (int e = tid; e < GT * D; e += 128) {
-    const int t = e / D, d = e - t * D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, red_m[w][t]);
-    float Lsum = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float mw = red_m[w][t];
-        const float wt = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
-        Lsum = fmaf(wt, red_l[w][t], Lsum);
-        O = fmaf(wt, red_o[w][t][d], O);
+        for (int j = 0; j < D / 8; ++j) *reinterpret_cast<float2*>(dw + 8 * j + 2 * tq) = make_float2(o[j][0], o[j][1]);
       }
-    }
-    const long long slot = (static_cast<long long>(n) * Hq + h0 + t) * max_splits + c;
-    part_o[slot * D + d] = O;
-    if (d == 0) {
-      part_ml[slot * 2] = M;
-      part_ml[slot * 2 + 1] = Lsum;
+      named_barrier_arrive(1, 128);
+    } else {
+      named_barrier(1, 128);
+      if (head) {
+        float M = mrow;
+#pragma unroll
+        for (int w = 0; w < 3; ++w) M = fmaxf(M, dep_m[w * 4 + gq]);
+        float e0 = 0.f, ew[3] = {0.f, 0.f, 0.f};
+        if (M != -INFINITY) {
+          e0 = mrow == -INFINITY ? 0.f : fast_exp2(mrow - M);
+#pragma unroll
+          for (int w = 0; w < 3; ++w) {
+            const float mw = dep_m[w * 4 + gq];
+            ew[w] = mw == -INFINITY ? 0.f : fast_exp2(mw - M);
+          }
+        }
+        float Lsum = e0 * lrow;
+#pragma unroll
+        for (int w = 0; w < 3; ++w) Lsum = fmaf(ew[w], dep_l[w * 4 + gq], Lsum);
+        const long long slot = (static_cast<long long>(it.n) * Hq + it.h0 + gq) * max_splits + it.c;
+        float* dst = part_o + slot * D;
+#pragma unroll
+        for (int j = 0; j < D / 8; ++j) {
+          float a0 = e0 * o[j][0], a1 = e0 * o[j][1];
+#pragma unroll
+          for (int w = 0; w < 3; ++w) {
+            const float2 y = *reinterpret_cast<const float2*>(dep + (w * GT + gq) * D + 8 * j + 2 * tq);
+            a0 = fmaf(ew[w], y.x, a0);
+            a1 = fmaf(ew[w], y.y, a1);
+          }
+          *reinterpret_cast<float2*>(dst + 8 * j + 2 * tq) = make_float2(a0, a1);
+        }
+        if (tq == 0) {
+          part_ml[slot * 2] = M;
+          part_ml[slot * 2 + 1] = Lsum;
+        }
+      }
+      named_barrier_arrive(2, 128);
     }
   }
+  if (warp > 0 && qi > 0) named_barrier(2, 128);  // pairs with warp 0's arrival for the last item
 }
 
 template <int D>
@@ -346,22 +426,30 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
   float acc[DPL];
 #pragma unroll
   for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-  for (int c = 0; c < C; ++c) {
-    const float wc = __shfl_sync(0xffffffffu, c < 32 ? w0 : w1, c & 31);
-    if (wc != 0.f) {
+  // eight partials per round, their loads all issued before the first is used
+  for (int c0 = 0; c0 < C; c0 += 8) {
+    float x[8][DPL], wv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int c = c0 + u;
+      wv[u] = __shfl_sync(0xffffffffu, c < 32 ? w0 : w1, c & 31);
       const float* src = part_o + (slot0 + c) * D + lane * DPL;
       if constexpr (DPL == 4) {
-        const float4 x = *reinterpret_cast<const float4*>(src);
-        acc[0] = fmaf(wc, x.x, acc[0]);
-        acc[1] = fmaf(wc, x.y, acc[1]);
-        acc[2] = fmaf(wc, x.z, acc[2]);
-        acc[3] = fmaf(wc, x.w, acc[3]);
+        const float4 y = c < C ? *reinterpret_cast<const float4*>(src) : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[u][0] = y.x;
+        x[u][1] = y.y;
+        x[u][2] = y.z;
+        x[u][3] = y.w;
       } else {
-        const float2 x = *reinterpret_cast<const float2*>(src);
-        acc[0] = fmaf(wc, x.x, acc[0]);
-        acc[1] = fmaf(wc, x.y, acc[1]);
+        const float2 y = c < C ? *reinterpret_cast<const float2*>(src) : make_float2(0.f, 0.f);
+        x[u][0] = y.x;
+        x[u][1] = y.y;
       }
     }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[e] = fmaf(wv[u], x[u][e], acc[e]);
   }
   const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
   uint16_t* dst = o + (static_cast<long long>(n) * Hq + h) * D + lane * DPL;
@@ -385,7 +473,14 @@ cudaError_t launch_split(const DecodeProblem& p, const void* q, const void* k, c
   cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, GT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.max_splits, p.Hkv * npass, p.N);
+  // a persistent grid: kDecCtasPerSm CTAs per SM, capped by the number of item slots
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const long long n_slots = static_cast<long long>(p.N) * p.Hkv * npass * p.max_splits;
+  const unsigned grid = static_cast<unsigned>(std::min<long long>(n_slots, static_cast<long long>(sms) * kDecCtasPerSm));
   {
     LaunchScope ls("decode_split", st);
     decode_split_kernel<D, GT><<<grid, kDecThreads, C::kSmemBytes, st>>>(

@@ -70,6 +70,10 @@ static_assert(kDecStages % 4 == 0, "decode ring stages must be a multiple of the
 constexpr int kDecThreads = 160;          // four compute warps + one producer warp
 constexpr int kDecCtasPerSm = 3;
 constexpr int kDecMapRows = 0x7fffffff;   // nominal row extent of the K/V tensor maps
+// Up to this many streams, every CTA numbers the valid items densely (a prefix sum of the per-stream
+// item counts in shared memory), so the static round-robin hands each CTA the same number of items
+// to within one; above it, CTAs walk the slot space and skip the slots past a stream's split count.
+constexpr int kDecDenseMax = 256;
 
 template <int D>
 struct DecCfg {
@@ -84,7 +88,8 @@ struct DecCfg {
   static constexpr int kOffBar = kOffDep + 3 * 4 * D * 4;
   static constexpr int kNumBars = 2 * kDecStages + 4;       // full, empty, q_full[2], q_empty[2]
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;   // abort flag, then the deposits' (m, l)
-  static constexpr int kSmemBytes = kOffMisc + 16 + 2 * 3 * 4 * 4 + 1024;
+  static constexpr int kOffBase = kOffMisc + 16 + 2 * 3 * 4 * 4;  // dense item numbering, see below
+  static constexpr int kSmemBytes = kOffBase + (kDecDenseMax + 1) * 4 + 1024;
 };
 
 // One work item: the key chunk c of stream n for the query heads h0 .. h0 + GT - 1 of kv head g.
@@ -94,6 +99,39 @@ struct DecItem {
 
 // Item slot idx -> item; false for slots past the stream's split count. Slots are ordered chunk
 // index slowest, so the first chunks of every stream and kv head come first.
+// The item whose fields are (n, c, gi) -> it; L = the stream's length, C_n its split count.
+template <int GT>
+__device__ __forceinline__ void dec_item_fill(int n, int c, int gi, int start, int L, int C_n, int Hq, int Hkv,
+                                              DecItem& it) {
+  const int G = Hq / Hkv, npass = G / GT;
+  const int chunk = (L + C_n - 1) / C_n;
+  it.n = n;
+  it.c = c;
+  it.g = gi / npass;
+  it.h0 = it.g * G + (gi % npass) * GT;
+  it.start = start;
+  it.k0 = min(L, c * chunk);
+  it.k1 = min(L, it.k0 + chunk);
+  it.nblk = (it.k1 - it.k0 + kDecBlk - 1) / kDecBlk;
+}
+
+// Dense item k -> item, with base[n] = NG * (C_0 + ... + C_{n-1}) in shared memory (N + 1 entries):
+// stream n holds items base[n] .. base[n + 1] - 1, kv head group gi = r / C_n, chunk c = r % C_n.
+template <int GT>
+__device__ __forceinline__ void dec_item_dense(int k, int N, int Hq, int Hkv, const int* offsets, const int* base,
+                                               DecItem& it) {
+  int lo = 0, hi = N;  // largest n with base[n] <= k
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (base[mid] <= k) lo = mid; else hi = mid;
+  }
+  const int NG = Hkv * ((Hq / Hkv) / GT);
+  const int C_n = (base[lo + 1] - base[lo]) / NG;
+  const int r = k - base[lo];
+  const int start = offsets[lo];
+  dec_item_fill<GT>(lo, r % C_n, r / C_n, start, offsets[lo + 1] - start, C_n, Hq, Hkv, it);
+}
+
 template <int GT>
 __device__ __forceinline__ bool dec_item(long long idx, int N, int Hq, int Hkv, const int* offsets,
                                          const int* num_splits, int max_splits, DecItem& it) {
@@ -106,15 +144,7 @@ __device__ __forceinline__ bool dec_item(long long idx, int N, int Hq, int Hkv, 
   const int L = offsets[n + 1] - start;
   const int C_n = stream_splits(num_splits, n, L, max_splits);
   if (c >= C_n) return false;
-  const int chunk = (L + C_n - 1) / C_n;
-  it.n = n;
-  it.c = c;
-  it.g = gi / npass;
-  it.h0 = it.g * G + (gi % npass) * GT;
-  it.start = start;
-  it.k0 = min(L, c * chunk);
-  it.k1 = min(L, it.k0 + chunk);
-  it.nblk = (it.k1 - it.k0 + kDecBlk - 1) / kDecBlk;
+  dec_item_fill<GT>(n, c, gi, start, L, C_n, Hq, Hkv, it);
   return true;
 }
 
@@ -153,9 +183,30 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
   float* dep_m = reinterpret_cast<float*>(smem + C::kOffMisc + 16);  // [3][4]
   float* dep_l = dep_m + 12;                                         // [3][4]
 
-  const int G = Hq / Hkv, npass = G / GT;
-  const long long n_slots = static_cast<long long>(N) * Hkv * npass * max_splits;
+  const int G = Hq / Hkv, npass = G / GT, NG = Hkv * npass;
+  const long long n_slots = static_cast<long long>(N) * NG * max_splits;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // dense numbering of the valid items (up to kDecDenseMax streams): warp 0 scans the per-stream
+  // item counts 32 streams at a time
+  int* base = reinterpret_cast<int*>(smem + C::kOffBase);
+  const bool dense = N <= kDecDenseMax;
+  if (dense && warp == 0) {
+    int run = 0;
+    for (int n0 = 0; n0 < N; n0 += 32) {
+      const int n = n0 + lane;
+      int cnt = 0;
+      if (n < N) cnt = NG * stream_splits(num_splits, n, offsets[n + 1] - offsets[n], max_splits);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (n < N) base[n] = run + incl - cnt;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) base[N] = run;
+  }
   if (tid == 0) {
     for (int s = 0; s < kDecStages; ++s) {
       mbar_init(full + s, 1);
@@ -169,6 +220,15 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
     fence_mbar_init();
   }
   __syncthreads();
+  const long long n_iter = dense ? base[N] : n_slots;  // items (dense) or slots (sparse)
+  // item number i of the walk -> item; false for a sparse slot past its stream's split count
+  auto next_item = [&](long long i, DecItem& it) -> bool {
+    if (dense) {
+      dec_item_dense<GT>(static_cast<int>(i), N, Hq, Hkv, offsets, base, it);
+      return true;
+    }
+    return dec_item<GT>(i, N, Hq, Hkv, offsets, num_splits, max_splits, it);
+  };
 
   if (warp == 4) {
     // ---------------------------------------------------------------- producer
@@ -177,9 +237,9 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
     long long gb = 0;  // ring position: blocks issued so far
     int qi = 0;        // items started so far
     bool ok = true;
-    for (long long idx = blockIdx.x; ok && idx < n_slots; idx += gridDim.x) {
+    for (long long idx = blockIdx.x; ok && idx < n_iter; idx += gridDim.x) {
       DecItem it;
-      if (!dec_item<GT>(idx, N, Hq, Hkv, offsets, num_splits, max_splits, it)) continue;
+      if (!next_item(idx, it)) continue;
       if (lane == 0) {  // the item's GT query rows (contiguous) into query buffer qi % 2
         ok = mbar_wait(q_empty + (qi & 1), ((qi >> 1) & 1) ^ 1, abort, status);
         if (ok) {
@@ -253,9 +313,9 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
   long long gb = 0;  // ring position of the current item's first block
   int qi = 0;
   bool ok = true;    // false once a wait has failed: the warp then only keeps the barrier protocol
-  for (long long idx = blockIdx.x; idx < n_slots; idx += gridDim.x) {
+  for (long long idx = blockIdx.x; idx < n_iter; idx += gridDim.x) {
     DecItem it;
-    if (!dec_item<GT>(idx, N, Hq, Hkv, offsets, num_splits, max_splits, it)) continue;
+    if (!next_item(idx, it)) continue;
     // this item's query rows (bf16) in shared memory; each block reads its Q fragments from there
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(q_full + (qi & 1), (qi >> 1) & 1, abort, status)) != 0;
     const uint32_t* qrow = reinterpret_cast<const uint32_t*>(sQ + (qi & 1) * C::kQBuf) + (head ? gq : 0) * (D / 2);

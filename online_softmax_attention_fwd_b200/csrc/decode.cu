@@ -116,7 +116,9 @@ __device__ __forceinline__ void dec_item_fill(int n, int c, int gi, int start, i
 }
 
 // Dense item k -> item, with base[n] = NG * (C_0 + ... + C_{n-1}) in shared memory (N + 1 entries):
-// stream n holds items base[n] .. base[n + 1] - 1, kv head group gi = r / C_n, chunk c = r % C_n.
+// stream n holds items base[n] .. base[n + 1] - 1, chunk c = r / NG, kv head group gi = r % NG. The
+// kv heads of one chunk are consecutive items, so neighbouring CTAs read the same cache rows at
+// about the same time (a row holds every kv head's keys side by side).
 template <int GT>
 __device__ __forceinline__ void dec_item_dense(int k, int N, int Hq, int Hkv, const int* offsets, const int* base,
                                                DecItem& it) {
@@ -129,7 +131,7 @@ __device__ __forceinline__ void dec_item_dense(int k, int N, int Hq, int Hkv, co
   const int C_n = (base[lo + 1] - base[lo]) / NG;
   const int r = k - base[lo];
   const int start = offsets[lo];
-  dec_item_fill<GT>(lo, r % C_n, r / C_n, start, offsets[lo + 1] - start, C_n, Hq, Hkv, it);
+  dec_item_fill<GT>(lo, r / NG, r % NG, start, offsets[lo + 1] - start, C_n, Hq, Hkv, it);
 }
 
 template <int GT>

@@ -485,6 +485,27 @@ def run_ours(args):
     return 0 if status == 0 else 1
 
 
+def run_case(name):
+    """One launch of each kernel of a workload and nothing else (a small command for ncu captures):
+    `prefill` = the 4k GQA causal forward and backward, `decode` = the 48-stream split-KV decode."""
+    import online_softmax_attention_fwd_b200 as attn
+    from online_softmax_attention_fwd_b200 import workloads as W
+    dev = torch.device("cuda")
+    if name == "prefill":
+        w = W.gqa_prefill_4k("A")
+        q, k, v, do = (t.to(dev) for t in (w.q, w.k, w.v, w.do))
+        o, lse = attn.fwd(q, k, v, causal=True, scale=w.scale)
+        attn.bwd(q, k, v, o, lse, do, causal=True, scale=w.scale)
+    else:
+        wd = W.decode48()
+        q, k, v, off = (t.to(dev) for t in (wd.q, wd.k, wd.v, wd.offsets))
+        attn.decode(q, k, v, off, scale=wd.scale)
+    torch.cuda.synchronize()
+    status = attn.device_status()
+    print(json.dumps({"case": name, "device_status": status}))
+    return 0 if status == 0 else 1
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -493,7 +514,11 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--case", choices=["prefill", "decode"],
+                    help="run one launch of each kernel of this workload and exit (for profilers)")
     args = ap.parse_args()
+    if args.case:
+        return run_case(args.case)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":

@@ -39,6 +39,8 @@
 // and MMA issuer (one elected lane of a converged warp). Every wait is bounded.
 #include <math.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tma_host.h"
@@ -481,74 +483,90 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Delta = rowsum(dO * O), lse2 = lse * log2(e) (+inf for rows that see no key), dQ accumulator = 0;
-// rows Sq .. Sq_pad - 1 are padding (lse2 = +inf, Delta = 0, accumulator 0). One warp per
-// (b, i, h) row of the padded range.
+// rows Sq .. Sq_pad - 1 are padding (lse2 = +inf, Delta = 0). A row (b, i, h) of the padded range is
+// D / 8 lanes, one 16-byte piece of O and dO each; a warp keeps four groups of rows in flight.
 template <int D>
-__global__ void __launch_bounds__(128) bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                                                        const float* __restrict__ lse, float* __restrict__ lse2,
                                                        float* __restrict__ delta, float* __restrict__ dq_acc, int B,
                                                        int Hq, int Sq, int Sq_pad) {
-  constexpr int DPL = D / 32;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long row = static_cast<long long>(blockIdx.x) * 4 + warp;  // (b, i, h) over Sq_pad, h fastest
-  if (row >= static_cast<long long>(B) * Sq_pad * Hq) return;
-  const int h = static_cast<int>(row % Hq);
-  const int i = static_cast<int>((row / Hq) % Sq_pad);
-  const int b = static_cast<int>(row / (static_cast<long long>(Hq) * Sq_pad));
-  float s = 0.f;
-  if (i < Sq) {
-    const long long base = ((static_cast<long long>(b) * Sq + i) * Hq + h) * D + lane * DPL;
-    if constexpr (DPL == 4) {
-      const uint2 x = *reinterpret_cast<const uint2*>(o + base);
-      const uint2 y = *reinterpret_cast<const uint2*>(dout + base);
-      s = bf16_lo(x.x) * bf16_lo(y.x) + bf16_hi(x.x) * bf16_hi(y.x) + bf16_lo(x.y) * bf16_lo(y.y) +
-          bf16_hi(x.y) * bf16_hi(y.y);
-    } else {
-      const uint32_t x = *reinterpret_cast<const uint32_t*>(o + base);
-      const uint32_t y = *reinterpret_cast<const uint32_t*>(dout + base);
-      s = bf16_lo(x) * bf16_lo(y) + bf16_hi(x) * bf16_hi(y);
+  constexpr int LPR = D / 8;     // lanes per row
+  constexpr int RPW = 32 / LPR;  // rows per warp instruction
+  constexpr int U = 4;           // row groups in flight per warp
+  const long long rows = static_cast<long long>(B) * Sq_pad * Hq;  // (b, i, h), h fastest
+  const int lane = threadIdx.x & 31, sub = lane / LPR, cl = lane % LPR;
+  const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long r0 = gw * RPW * U; r0 < rows; r0 += nw * RPW * U) {
+    uint4 x[U], y[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long row = r0 + u * RPW + sub;
+      const int h = static_cast<int>(row % Hq);
+      const int i = static_cast<int>((row / Hq) % Sq_pad);
+      const long long b = row / (static_cast<long long>(Hq) * Sq_pad);
+      x[u] = y[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (row < rows && i < Sq) {
+        const long long base = ((b * Sq + i) * Hq + h) * D + cl * 8;
+        x[u] = *reinterpret_cast<const uint4*>(o + base);
+        y[u] = *reinterpret_cast<const uint4*>(dout + base);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t xs[4] = {x[u].x, x[u].y, x[u].z, x[u].w}, ys[4] = {y[u].x, y[u].y, y[u].z, y[u].w};
+      float sacc = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc += bf16_lo(xs[e]) * bf16_lo(ys[e]) + bf16_hi(xs[e]) * bf16_hi(ys[e]);
+#pragma unroll
+      for (int off = LPR / 2; off > 0; off >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, off);
+      const long long row = r0 + u * RPW + sub;
+      if (cl == 0 && row < rows) {
+        const int h = static_cast<int>(row % Hq);
+        const int i = static_cast<int>((row / Hq) % Sq_pad);
+        const long long b = row / (static_cast<long long>(Hq) * Sq_pad);
+        const long long li = (b * Hq + h) * Sq_pad + i;
+        delta[li] = sacc;
+        const float l = i < Sq ? lse[(b * Hq + h) * Sq + i] : -INFINITY;
+        lse2[li] = (l == -INFINITY) ? INFINITY : l * kLog2e;
+      }
     }
   }
-  // zero D accumulator values per row: together the rows cover the whole accumulator, whatever
-  // its internal order
-  const long long abase = row * D + lane * DPL;
-  if constexpr (DPL == 4)
-    *reinterpret_cast<float4*>(dq_acc + abase) = make_float4(0.f, 0.f, 0.f, 0.f);
-  else
-    *reinterpret_cast<float2*>(dq_acc + abase) = make_float2(0.f, 0.f);
-  s = warp_sum(s);
-  if (lane == 0) {
-    const long long li = (static_cast<long long>(b) * Hq + h) * Sq_pad + i;
-    delta[li] = s;
-    const float l = i < Sq ? lse[(static_cast<long long>(b) * Hq + h) * Sq + i] : -INFINITY;
-    lse2[li] = (l == -INFINITY) ? INFINITY : l * kLog2e;
-  }
+  // the whole accumulator (rows x D values, whatever its internal order) to zero
+  const long long n4 = rows * D / 4;
+  for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < n4;
+       t += static_cast<long long>(gridDim.x) * blockDim.x)
+    reinterpret_cast<float4*>(dq_acc)[t] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// dQ = scale * accumulator -> bf16. A thread takes two adjacent head-dim columns of one group of
-// four query rows (two float4 of the interleaved accumulator) and writes a bf16 pair to each of
-// the four rows that exist.
+// dQ = scale * accumulator -> bf16. A thread takes four adjacent head-dim columns of one group of
+// four query rows (four consecutive float4 of the interleaved accumulator, 64 bytes), transposes
+// them and writes four bf16 to each of the four rows that exist; a warp covers 128 columns.
 __global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const float* __restrict__ acc,
                                                              uint16_t* __restrict__ dq, int B, int Hq, int Sq,
                                                              int Sq_pad, int D, float scale) {
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int half_d = D / 2, groups = Sq_pad / 4;
-  if (i >= static_cast<long long>(B) * Hq * groups * half_d) return;
-  const int dp = static_cast<int>(i % half_d);
-  long long t = i / half_d;
+  const int qd = D / 4, groups = Sq_pad / 4;
+  if (i >= static_cast<long long>(B) * Hq * groups * qd) return;
+  const int d4 = static_cast<int>(i % qd);
+  long long t = i / qd;
   const int g4 = static_cast<int>(t % groups);
   t /= groups;
   const int h = static_cast<int>(t % Hq);
   const long long b = t / Hq;
-  const float4* src = reinterpret_cast<const float4*>(acc) + ((b * Hq + h) * groups + g4) * D + 2 * dp;
-  const float4 x = src[0];  // column 2 dp, rows 4 g4 .. 4 g4 + 3
-  const float4 y = src[1];  // column 2 dp + 1
-  const float xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+  const float4* src = reinterpret_cast<const float4*>(acc) + ((b * Hq + h) * groups + g4) * D + 4 * d4;
+  const float4 c0 = src[0], c1 = src[1], c2 = src[2], c3 = src[3];  // columns 4 d4 + k, rows 4 g4 .. + 3
+  const float r0[4] = {c0.x, c0.y, c0.z, c0.w}, r1[4] = {c1.x, c1.y, c1.z, c1.w};
+  const float r2[4] = {c2.x, c2.y, c2.z, c2.w}, r3[4] = {c3.x, c3.y, c3.z, c3.w};
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     const int q = 4 * g4 + e;
-    if (q < Sq)
-      *reinterpret_cast<uint32_t*>(dq + ((b * Sq + q) * Hq + h) * D + 2 * dp) = pack_bf16(xs[e] * scale, ys[e] * scale);
+    if (q < Sq) {
+      uint2 w;
+      w.x = pack_bf16(r0[e] * scale, r1[e] * scale);
+      w.y = pack_bf16(r2[e] * scale, r3[e] * scale);
+      *reinterpret_cast<uint2*>(dq + ((b * Sq + q) * Hq + h) * D + 4 * d4) = w;
+    }
   }
 }
 
@@ -573,7 +591,9 @@ cudaError_t launch_bwd_sm100_d(const Problem& p, const void* q, const void* k, c
 
   {
     LaunchScope ls("bwd_prep", st);
-    bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, st>>>(
+    // rows / (8 warps x 2 or 4 rows x 4 groups) blocks, grid-strided
+    const unsigned blocks = static_cast<unsigned>(std::min<size_t>((rows + 63) / 64, 1u << 20));
+    bwd_prep_kernel<D><<<blocks, 256, 0, st>>>(
         static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, lse2, delta, dq_acc, p.B, p.Hq,
         p.Sq, Sq_pad);
   }
@@ -606,7 +626,7 @@ cudaError_t launch_bwd_sm100_d(const Problem& p, const void* q, const void* k, c
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
-  const long long n_conv = static_cast<long long>(p.B) * p.Hq * (Sq_pad / 4) * (D / 2);
+  const long long n_conv = static_cast<long long>(p.B) * p.Hq * (Sq_pad / 4) * (D / 4);
   {
     LaunchScope ls("bwd_dq_convert", st);
     bwd_dq_convert_kernel<<<static_cast<unsigned>((n_conv + 255) / 256), 256, 0, st>>>(

@@ -66,8 +66,11 @@ struct BwdCfg {
   static constexpr int kOffBar = kOffDS + 2 * kAtom;
   static constexpr int kNumBars = 1 + 2 * kStages + 9;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kOffRow = kOffMisc + 64;              // lse2 and Delta of the current tile
+  // lse2 and Delta of the current tile, read as float4: 16-byte aligned whatever the barrier count
+  static constexpr int kOffRow = (kOffMisc + 64 + 15) & ~15;
   static constexpr int kSmemBytes = kOffRow + 2 * kBM * 4 + 1024;
+  static_assert(kOffRow % 16 == 0, "the lse2 / Delta rows are read with 16-byte loads");
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
 };
 

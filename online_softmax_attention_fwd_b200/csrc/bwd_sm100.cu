@@ -297,6 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------------ score warps (row = key)
+    griddep_wait();  // lse2 and Delta come from bwd_prep
     const int t = threadIdx.x;  // TMEM lane == key row in the tile
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t tS = tmem + lane_addr + C::kColS, tDP = tmem + lane_addr + C::kColDP;
@@ -444,6 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ dQ drain (warps 4-7)
+    griddep_wait();  // bwd_prep has cleared the accumulator
     // Thread e holds TMEM lane e = head-dim column d of dQ^T; for each group of four query rows the
     // warp's 32 lanes add 32 consecutive columns x 4 rows (512 contiguous bytes) into the
     // interleaved accumulator.
@@ -483,6 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  griddep_launch_dependents();
 }
 
 // Delta = rowsum(dO * O), lse2 = lse * log2(e) (+inf for rows that see no key), dQ accumulator = 0;
@@ -548,6 +551,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
 __global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const float* __restrict__ acc,
                                                              uint16_t* __restrict__ dq, int B, int Hq, int Sq,
                                                              int Sq_pad, int D, float scale) {
+  griddep_wait();  // the accumulator is complete
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int qd = D / 4, groups = Sq_pad / 4;
   if (i >= static_cast<long long>(B) * Hq * groups * qd) return;
@@ -624,17 +628,19 @@ cudaError_t launch_bwd_sm100_d(const Problem& p, const void* q, const void* k, c
   dim3 grid(p.Hkv * p.B, (p.Sk + kBN - 1) / kBN);
   {
     LaunchScope ls("bwd_sm100", st);
-    bwd_sm100_kernel<D><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, mdo, a);
+    e = launch_dependent(bwd_sm100_kernel<D>, grid, dim3(kThreads), C::kSmemBytes, st, mq, mk, mv, mdo, a);
   }
+  if (e != cudaSuccess) return e;
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
   const long long n_conv = static_cast<long long>(p.B) * p.Hq * (Sq_pad / 4) * (D / 4);
   {
     LaunchScope ls("bwd_dq_convert", st);
-    bwd_dq_convert_kernel<<<static_cast<unsigned>((n_conv + 255) / 256), 256, 0, st>>>(
-        dq_acc, static_cast<uint16_t*>(dq), p.B, p.Hq, p.Sq, Sq_pad, D, p.scale);
+    e = launch_dependent(bwd_dq_convert_kernel, dim3(static_cast<unsigned>((n_conv + 255) / 256)), dim3(256), 0, st,
+                         dq_acc, static_cast<uint16_t*>(dq), p.B, p.Hq, p.Sq, Sq_pad, D, p.scale);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -449,6 +449,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
     }
   }
   if (warp > 0 && qi > 0) named_barrier(2, 128);  // pairs with warp 0's arrival for the last item
+  griddep_launch_dependents();
 }
 
 template <int D>
@@ -459,6 +460,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
                                                              int N, int Hq, uint16_t* __restrict__ o,
                                                              float* __restrict__ lse) {
   constexpr int DPL = D / 32;
+  griddep_wait();  // the split kernel's partial triples
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long gw = static_cast<long long>(blockIdx.x) * 4 + warp;
   if (gw >= static_cast<long long>(N) * Hq) return;
@@ -466,7 +468,26 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
   const int L = offsets[n + 1] - offsets[n];
   const int C = stream_splits(num_splits, n, L, max_splits);
   const long long slot0 = (static_cast<long long>(n) * Hq + h) * max_splits;
-  // lane c holds chunk c and chunk c + 32 (max_splits <= 64)
+  // The first 16 partial rows are loaded before anything else, so their loads and those of the
+  // (m, l) pairs are in flight together; lane c holds the pair of chunk c and c + 32 (max_splits
+  // <= 64).
+  constexpr int kFirst = 16;
+  float x[kFirst][DPL];
+#pragma unroll
+  for (int c = 0; c < kFirst; ++c) {
+    const float* src = part_o + (slot0 + c) * D + lane * DPL;
+    if constexpr (DPL == 4) {
+      const float4 y = c < C ? *reinterpret_cast<const float4*>(src) : make_float4(0.f, 0.f, 0.f, 0.f);
+      x[c][0] = y.x;
+      x[c][1] = y.y;
+      x[c][2] = y.z;
+      x[c][3] = y.w;
+    } else {
+      const float2 y = c < C ? *reinterpret_cast<const float2*>(src) : make_float2(0.f, 0.f);
+      x[c][0] = y.x;
+      x[c][1] = y.y;
+    }
+  }
   float m0 = -INFINITY, l0 = 0.f, m1 = -INFINITY, l1 = 0.f;
   if (lane < C) {
     const float2 ml = *reinterpret_cast<const float2*>(part_ml + (slot0 + lane) * 2);
@@ -488,30 +509,27 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
   float acc[DPL];
 #pragma unroll
   for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-  // eight partials per round, their loads all issued before the first is used
-  for (int c0 = 0; c0 < C; c0 += 8) {
-    float x[8][DPL], wv[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+  for (int c = 0; c < kFirst; ++c) {
+    const float wc = __shfl_sync(0xffffffffu, w0, c);  // 0 for c >= C
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[e] = fmaf(wc, x[c][e], acc[e]);
+  }
+  // any further partials, four per round
+  for (int c0 = kFirst; c0 < C; c0 += 4) {
+    float y4[4][DPL], wv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
       const int c = c0 + u;
       wv[u] = __shfl_sync(0xffffffffu, c < 32 ? w0 : w1, c & 31);
       const float* src = part_o + (slot0 + c) * D + lane * DPL;
-      if constexpr (DPL == 4) {
-        const float4 y = c < C ? *reinterpret_cast<const float4*>(src) : make_float4(0.f, 0.f, 0.f, 0.f);
-        x[u][0] = y.x;
-        x[u][1] = y.y;
-        x[u][2] = y.z;
-        x[u][3] = y.w;
-      } else {
-        const float2 y = c < C ? *reinterpret_cast<const float2*>(src) : make_float2(0.f, 0.f);
-        x[u][0] = y.x;
-        x[u][1] = y.y;
-      }
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) y4[u][e] = c < C ? src[e] : 0.f;
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
+    for (int u = 0; u < 4; ++u)
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) acc[e] = fmaf(wv[u], x[u][e], acc[e]);
+      for (int e = 0; e < DPL; ++e) acc[e] = fmaf(wv[u], y4[u][e], acc[e]);
   }
   const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
   uint16_t* dst = o + (static_cast<long long>(n) * Hq + h) * D + lane * DPL;
@@ -579,8 +597,10 @@ cudaError_t launch_decode_d(const DecodeProblem& p, const void* q, const void* k
   const long long warps = static_cast<long long>(p.N) * p.Hq;
   {
     LaunchScope ls("decode_combine", st);
-    decode_combine_kernel<D><<<static_cast<unsigned>((warps + 3) / 4), 128, 0, st>>>(
-        part_o, part_ml, offsets, num_splits, p.max_splits, p.N, p.Hq, static_cast<uint16_t*>(o), lse);
+    const cudaError_t e2 =
+        launch_dependent(decode_combine_kernel<D>, dim3(static_cast<unsigned>((warps + 3) / 4)), dim3(128), 0, st,
+                         part_o, part_ml, offsets, num_splits, p.max_splits, p.N, p.Hq, static_cast<uint16_t*>(o), lse);
+    if (e2 != cudaSuccess) return e2;
   }
   return cudaGetLastError();
 }

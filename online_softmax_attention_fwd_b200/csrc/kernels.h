@@ -25,6 +25,26 @@ class LaunchScope {
   cudaStream_t st_;
   int slot_;
 };
+// Launch of a kernel that follows another kernel of the same call on the same stream, with
+// programmatic dependent launch: its CTAs may be scheduled while the previous kernel's last CTAs
+// finish, and it must execute griddep_wait() before it touches anything the previous kernel
+// writes (or anything written before that kernel, which the previous kernel waited for).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Device pointer of the library's status word on the current device (nullptr if unavailable).
 int* device_status_ptr();
 

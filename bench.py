@@ -488,6 +488,7 @@ def run_ours(args):
 def run_case(name):
     """One launch of each kernel of a workload and nothing else (a small command for ncu captures):
     `prefill` = the 4k GQA causal forward and backward, `decode` = the 48-stream split-KV decode."""
+    import torch
     import online_softmax_attention_fwd_b200 as attn
     from online_softmax_attention_fwd_b200 import workloads as W
     dev = torch.device("cuda")

@@ -9,7 +9,13 @@
 // The two contractions are dense, so they run as tcgen05.mma with fp32 accumulators in tensor
 // memory; the row statistics run on the CUDA cores, one thread per row.
 //
-// A CTA owns two 128-row query tiles of one head and streams each 128-key K/V block once for both.
+// The grid is persistent (one CTA per SM). A work item is two 128-row query tiles of one head, and
+// the CTA streams each 128-key K/V block once for both. Items are sorted longest first (under a
+// causal mask the last tile pairs see the most keys) and dealt to the CTAs in snake order. Across
+// items the K/V ring runs on without a pause. The next item's Q is loaded as soon as the current
+// item's last S is complete, and a tile's epilogue overlaps the next item's first S; the first P V
+// of an item waits only until that epilogue has read O out of TMEM (barrier o_free).
+// Otherwise a CTA works on one item as follows.
 // TMEM holds, per tile, S (128 columns) and O (128 columns): 512 in all. The softmax writes P as
 // bf16 back over the first 64 columns of its own S, and P V reads it from there (A operand in
 // TMEM), so P never goes through shared memory. Every MMA is 128 wide in N, which keeps the tensor
@@ -31,6 +37,8 @@
 // Shared-memory tiles use the 128-byte swizzle: Q and K are K-major (rows of 64 bf16 = 128 B), V is
 // read as an MN-major operand (its head dim is contiguous). Every wait is bounded (common.cuh).
 #include <math.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -60,7 +68,7 @@ struct FwdCfg {
   static constexpr int kOffK = kOffQ + 2 * kTileBytes;                 // [K stages]
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;          // [V stages]
   static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
-  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 4 + 2 + 1;
+  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 4 + 2 + 2 + 1 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + slack for 1024-byte alignment
   // TMEM: S (and P over its first 64 columns) of tile t at 128 t; O of tile t at 256 + 128 t.
@@ -95,6 +103,13 @@ __device__ __forceinline__ int tile_blocks(const FwdArgs& a, int qs) {
   return kv_end > 0 ? (kv_end + kBN - 1) / kBN : 0;
 }
 
+// Work item k of CTA c under the snake order (round r = k: CTAs c = 0 .. G-1 left to right on even
+// rounds, right to left on odd ones) over items sorted longest first; -1 past the end.
+__device__ __forceinline__ int fwd_item_index(int k, int c, int G, int n_items) {
+  const int i = k * G + ((k & 1) ? (G - 1 - c) : c);
+  return i < n_items ? i : -1;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -113,24 +128,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_empty = v_full + C::kVStages;
   uint64_t* s_full = v_empty + C::kVStages;  // [tile]
   uint64_t* p_full = s_full + 2;             // [tile][half]: P of keys 0-63 / 64-127 in TMEM
-  uint64_t* o_done = p_full + 4;             // [tile]: every P V of the tile is complete
-  uint64_t* drain = o_done + 2;
+  uint64_t* o_done = p_full + 4;             // [tile]: every P V of the tile's item is complete
+  uint64_t* o_free = o_done + 2;             // [tile]: the epilogue has read O out of TMEM
+  uint64_t* q_empty = o_free + 2;            // the item's last S = Q K^T is complete
+  uint64_t* drain = q_empty + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // blockIdx.y walks the tile pairs from the last (longest under a causal mask) to the first, and
-  // blockIdx.x, which varies fastest in launch order, covers every (batch, head): the longest tiles
-  // of all heads start first.
-  const int pair = a.n_pairs - 1 - static_cast<int>(blockIdx.y);
-  const int h = static_cast<int>(blockIdx.x) % a.Hq, b = static_cast<int>(blockIdx.x) / a.Hq;
-  const int g = h / (a.Hq / a.Hkv);
-  const int q0 = pair * 2 * kBM;
-  const int n0 = tile_blocks(a, q0), n1 = tile_blocks(a, q0 + kBM);
-  const int nmax = max(n0, n1);
+  const int BH = a.B * a.Hq;
+  const int n_items = BH * a.n_pairs;
+  const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
+  // item i: tile pair n_pairs - 1 - i / BH (the longest pairs first under a causal mask), (b, h) = i % BH
+  auto item_of = [&](int i, int& b, int& h, int& q0, int& n0, int& n1) {
+    const int bh = i % BH, pair = a.n_pairs - 1 - i / BH;
+    b = bh / a.Hq;
+    h = bh % a.Hq;
+    q0 = pair * 2 * kBM;
+    n0 = tile_blocks(a, q0);
+    n1 = tile_blocks(a, q0 + kBM);
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < C::kKStages; ++s) {
       mbar_init(k_full + s, 1);
       mbar_init(k_empty + s, 1);
@@ -144,6 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(p_full + 2 * t, 4);
       mbar_init(p_full + 2 * t + 1, 4);
       mbar_init(o_done + t, 1);
+      mbar_init(o_free + t, 4);
     }
     mbar_init(drain, 1);
     *abort = 0;
@@ -165,94 +187,133 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 8) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0 && nmax > 0) {
+    if (lane == 0) {
       constexpr uint32_t kTx = kBM * D * 2;
-      mbar_arrive_expect_tx(q_full, (n0 > 0 ? kTx : 0u) + (n1 > 0 ? kTx : 0u));
+      long long kvb = 0;  // K/V blocks issued so far (ring position)
+      int qk = 0;         // items with any block so far
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int i = fwd_item_index(k, cta, G, n_items);
+        if (i < 0) break;
+        int b, h, q0, n0, n1;
+        item_of(i, b, h, q0, n0, n1);
+        const int nmax = max(n0, n1);
+        if (nmax == 0) continue;
+        const int g = h / (a.Hq / a.Hkv);
+        // this item's Q tiles once the previous item's last S has read the buffer
+        if (!mbar_wait(q_empty, (qk & 1) ^ 1, abort, a.status)) break;
+        mbar_arrive_expect_tx(q_full, (n0 > 0 ? kTx : 0u) + (n1 > 0 ? kTx : 0u));
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if ((t == 0 ? n0 : n1) == 0) continue;
+        for (int t = 0; t < 2; ++t) {
+          if ((t == 0 ? n0 : n1) == 0) continue;
 #pragma unroll
-        for (int at = 0; at < C::kAtoms; ++at)
-          tma_load_4d(sQ + t * C::kTileBytes + at * kAtom, &tmQ, q_full, at * 64, h, q0 + t * kBM, b);
-      }
-      int issued_k = 0, issued_v = 0;
-      for (int j = 0; j < nmax; ++j) {
-        const int sk = j % C::kKStages, sv = j % C::kVStages;
-        if (!mbar_wait(k_empty + sk, ((j / C::kKStages) & 1) ^ 1, abort, a.status)) break;
-        mbar_arrive_expect_tx(k_full + sk, kTx);
+          for (int at = 0; at < C::kAtoms; ++at)
+            tma_load_4d(sQ + t * C::kTileBytes + at * kAtom, &tmQ, q_full, at * 64, h, q0 + t * kBM, b);
+        }
+        ++qk;
+        for (int j = 0; j < nmax; ++j) {
+          const long long gj = kvb + j;
+          const int sk = static_cast<int>(gj % C::kKStages), sv = static_cast<int>(gj % C::kVStages);
+          if (!mbar_wait(k_empty + sk, static_cast<uint32_t>((gj / C::kKStages) & 1) ^ 1, abort, a.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(k_full + sk, kTx);
 #pragma unroll
-        for (int at = 0; at < C::kAtoms; ++at)
-          tma_load_4d(sK + sk * C::kTileBytes + at * kAtom, &tmK, k_full + sk, at * 64, g, j * kBN, b);
-        issued_k = j + 1;
-        if (!mbar_wait(v_empty + sv, ((j / C::kVStages) & 1) ^ 1, abort, a.status)) break;
-        mbar_arrive_expect_tx(v_full + sv, kTx);
+          for (int at = 0; at < C::kAtoms; ++at)
+            tma_load_4d(sK + sk * C::kTileBytes + at * kAtom, &tmK, k_full + sk, at * 64, g, j * kBN, b);
+          if (!mbar_wait(v_empty + sv, static_cast<uint32_t>((gj / C::kVStages) & 1) ^ 1, abort, a.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(v_full + sv, kTx);
 #pragma unroll
-        for (int at = 0; at < C::kAtoms; ++at)
-          tma_load_4d(sV + sv * C::kTileBytes + at * kAtom, &tmV, v_full + sv, at * 64, g, j * kBN, b);
-        issued_v = j + 1;
+          for (int at = 0; at < C::kAtoms; ++at)
+            tma_load_4d(sV + sv * C::kTileBytes + at * kAtom, &tmV, v_full + sv, at * 64, g, j * kBN, b);
+        }
+        kvb += nmax;
       }
       // Let every load this thread issued land before the CTA can exit. On the normal path the
       // consumers have already waited for each of them, so these return at once.
-      wait_drain(q_full, 0);
-      for (int j = max(0, issued_k - C::kKStages); j < issued_k; ++j)
-        wait_drain(k_full + j % C::kKStages, (j / C::kKStages) & 1);
-      for (int j = max(0, issued_v - C::kVStages); j < issued_v; ++j)
-        wait_drain(v_full + j % C::kVStages, (j / C::kVStages) & 1);
+      if (qk > 0) wait_drain(q_full, (qk - 1) & 1);
+      for (long long j = max(0ll, kvb - C::kKStages); j < kvb; ++j)
+        wait_drain(k_full + j % C::kKStages, static_cast<uint32_t>((j / C::kKStages) & 1));
+      for (long long j = max(0ll, kvb - C::kVStages); j < kvb; ++j)
+        wait_drain(v_full + j % C::kVStages, static_cast<uint32_t>((j / C::kVStages) & 1));
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
-    if (nmax > 0) {  // the whole warp runs the loop; one elected lane issues each MMA
-      constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, 0, 0);
-      constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, D, 0, 1);
-      // base descriptors, built once; each MMA only moves the start address
-      const uint64_t dQ0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
-      const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);
-      const uint64_t dV0 = sdesc_sw128(smem_u32(sV), kAtom, 1024);
-      const int nt[2] = {n0, n1};
-      bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort, a.status));
-      int k_ready = -1, v_ready = -1;  // last K / V block this warp has waited for
-      auto wait_k = [&](int jb) -> bool {
-        if (k_ready >= jb) return true;
-        k_ready = jb;
-        return __all_sync(0xffffffffu, mbar_wait(k_full + jb % C::kKStages, (jb / C::kKStages) & 1, abort, a.status)) != 0;
-      };
-      auto wait_v = [&](int jb) -> bool {
-        if (v_ready >= jb) return true;
-        v_ready = jb;
-        return __all_sync(0xffffffffu, mbar_wait(v_full + jb % C::kVStages, (jb / C::kVStages) & 1, abort, a.status)) != 0;
-      };
-      // S_t of block jb = Q_t K_jb^T
-      auto issue_s = [&](int t, int jb) {
-        tc_fence_after();
-        const uint64_t dK = sdesc_advance(dK0, (jb % C::kKStages) * C::kTileBytes);
-        const uint64_t dQ = sdesc_advance(dQ0, t * C::kTileBytes);
+    // the whole warp runs the loop; one elected lane issues each MMA
+    constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, 0, 0);
+    constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, D, 0, 1);
+    // base descriptors, built once; each MMA only moves the start address
+    const uint64_t dQ0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+    const uint64_t dV0 = sdesc_sw128(smem_u32(sV), kAtom, 1024);
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, a.status)) != 0;
+    };
+    long long kvb = 0;      // ring position of the item's first K/V block
+    long long k_ready = -1, v_ready = -1;  // last K / V block this warp has waited for
+    long long sb[2] = {0, 0};  // S blocks of each tile issued in earlier items
+    int ct[2] = {0, 0};        // earlier items in which each tile had blocks
+    int qk = 0;
+    bool ok = true;
+    auto wait_k = [&](long long gj) -> bool {
+      if (k_ready >= gj) return true;
+      k_ready = gj;
+      return wait_all(k_full + gj % C::kKStages, static_cast<uint32_t>((gj / C::kKStages) & 1));
+    };
+    auto wait_v = [&](long long gj) -> bool {
+      if (v_ready >= gj) return true;
+      v_ready = gj;
+      return wait_all(v_full + gj % C::kVStages, static_cast<uint32_t>((gj / C::kVStages) & 1));
+    };
+    // S_t of ring block gj = Q_t K^T
+    auto issue_s = [&](int t, long long gj) {
+      tc_fence_after();
+      const uint64_t dK = sdesc_advance(dK0, static_cast<uint32_t>(gj % C::kKStages) * C::kTileBytes);
+      const uint64_t dQ = sdesc_advance(dQ0, t * C::kTileBytes);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
-          umma_ss_warp(tmem + C::colS(t), sdesc_advance(dQ, off), sdesc_advance(dK, off), kIdescS, kk > 0);
-        }
-        umma_commit_warp(s_full + t);
-      };
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
+        umma_ss_warp(tmem + C::colS(t), sdesc_advance(dQ, off), sdesc_advance(dK, off), kIdescS, kk > 0);
+      }
+      umma_commit_warp(s_full + t);
+    };
+    for (int k = 0; ok; ++k) {
+      const int i = fwd_item_index(k, cta, G, n_items);
+      if (i < 0) break;
+      int b, h, q0, n0, n1;
+      item_of(i, b, h, q0, n0, n1);
+      const int nmax = max(n0, n1);
+      if (nmax == 0) continue;
+      const int nt[2] = {n0, n1};
+      if (!wait_all(q_full, qk & 1) || !wait_k(kvb)) break;
+      // S of block 0 for both tiles (over P of the previous item, whose P V was issued earlier)
+      for (int t = 0; t < 2; ++t)
+        if (nt[t] > 0) issue_s(t, kvb);
+      umma_commit_warp(k_empty + kvb % C::kKStages);
+      if (nmax == 1) umma_commit_warp(q_empty);  // this item's Q has been read by all its S
       // per block j and tile t: O_t += P_t V_j, then at once S_t of block j + 1 (it overwrites P_t in
       // TMEM; the P V that reads P_t was issued just before it and MMAs execute in order). The two
       // tiles' chains are independent, so the tensor pipe alternates between them.
-      if (ok && wait_k(0)) {
-        for (int t = 0; t < 2; ++t)
-          if (nt[t] > 0) issue_s(t, 0);
-        umma_commit_warp(k_empty);
-      } else {
-        ok = false;
-      }
       for (int j = 0; ok && j < nmax; ++j) {
+        const long long gj = kvb + j;
         for (int t = 0; t < 2; ++t) {
           if (j < nt[t]) {
-            const uint64_t dV = sdesc_advance(dV0, (j % C::kVStages) * C::kTileBytes);
+            // the first P V of the item overwrites O_t: the previous item's epilogue must have read it
+            if (j == 0 && ct[t] > 0 && !wait_all(o_free + t, (ct[t] - 1) & 1)) {
+              ok = false;
+              break;
+            }
+            const uint64_t dV = sdesc_advance(dV0, static_cast<uint32_t>(gj % C::kVStages) * C::kTileBytes);
             // P (bf16) is the A operand in TMEM, 16 keys = 8 columns per step; each half of the
             // block's keys goes as soon as the softmax has written its P
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-              if ((hf == 0 && !wait_v(j)) ||
-                  !__all_sync(0xffffffffu, mbar_wait(p_full + 2 * t + hf, j & 1, abort, a.status))) {
+              if ((hf == 0 && !wait_v(gj)) ||
+                  !wait_all(p_full + 2 * t + hf, static_cast<uint32_t>((sb[t] + j) & 1))) {
                 ok = false;
                 break;
               }
@@ -266,22 +327,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (j == nt[t] - 1) umma_commit_warp(o_done + t);
           }
           if (j + 1 < nt[t]) {
-            if (!wait_k(j + 1)) {
+            if (!wait_k(gj + 1)) {
               ok = false;
               break;
             }
-            issue_s(t, j + 1);
+            issue_s(t, gj + 1);
           }
         }
         if (!ok) break;
-        if (j + 1 < nmax) umma_commit_warp(k_empty + (j + 1) % C::kKStages);
-        umma_commit_warp(v_empty + j % C::kVStages);
+        if (j + 1 < nmax) umma_commit_warp(k_empty + (gj + 1) % C::kKStages);
+        if (j + 2 == nmax) umma_commit_warp(q_empty);  // the item's last S has been issued
+        umma_commit_warp(v_empty + gj % C::kVStages);
       }
-      // all MMAs issued by this warp complete before the CTA releases TMEM
-      umma_commit_warp(drain);
-      wait_drain(drain, 0);
-      __syncwarp();
+      if (!ok) break;
+      for (int t = 0; t < 2; ++t)
+        if (nt[t] > 0) {
+          sb[t] += nt[t];
+          ++ct[t];
+        }
+      kvb += nmax;
+      ++qk;
     }
+    // all MMAs issued by this warp complete before the CTA releases TMEM
+    umma_commit_warp(drain);
+    wait_drain(drain, 0);
+    __syncwarp();
   } else {
     // ------------------------------------------------------------------ softmax warpgroups
     const int t = warp >> 2;               // query tile of this warpgroup
@@ -289,128 +359,147 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_addr + C::colS(t);
     const uint32_t tO = tmem + lane_addr + C::colO(t);
-    const int n_kv = t == 0 ? n0 : n1;
-    const int qrow = q0 + t * kBM + row;
-    int row_limit = a.Sk - 1;  // largest visible key index for this row
-    if (a.causal) row_limit = min(row_limit, qrow + a.Sk - a.Sq);
-    float m = -INFINITY, l = 0.f;
-    bool ok = true;
     // every lane waits; the outcome is made warp-uniform before any warp-collective tcgen05 op
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
       const bool r = mbar_wait(bar, parity, abort, a.status);
       return __all_sync(0xffffffffu, r);
     };
-    for (int j = 0; j < n_kv; ++j) {
-      if (!wait_warp(s_full + t, j & 1)) {
-        ok = false;
-        break;
+    long long sb = 0;  // this tile's S blocks in earlier items
+    int ct = 0;        // earlier items in which this tile had blocks
+    bool ok = true;
+    for (int k = 0;; ++k) {
+      const int i = fwd_item_index(k, cta, G, n_items);
+      if (i < 0) break;
+      int b, h, q0, n0, n1;
+      item_of(i, b, h, q0, n0, n1);
+      const int n_kv = t == 0 ? n0 : n1;
+      const int qrow = q0 + t * kBM + row;
+      int row_limit = a.Sk - 1;  // largest visible key index for this row
+      if (a.causal) row_limit = min(row_limit, qrow + a.Sk - a.Sq);
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; ok && j < n_kv; ++j) {
+        if (!wait_warp(s_full + t, static_cast<uint32_t>((sb + j) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int kbase = j * kBN;
+        // the whole 128-column row of S in registers: one round trip to TMEM
+        uint32_t sr[kBN];
+  #pragma unroll
+        for (int c = 0; c < kBN; c += 16) tmem_ld16(tS + c, sr + c);
+        tmem_wait_ld();
+        if (kbase + kBN - 1 > row_limit) {  // the block crosses this row's last visible key
+  #pragma unroll
+          for (int c = 0; c < kBN; ++c)
+            if (kbase + c > row_limit) sr[c] = __float_as_uint(-INFINITY);
+        }
+        float mx8[8];  // eight independent max chains
+  #pragma unroll
+        for (int c = 0; c < 8; ++c) mx8[c] = __uint_as_float(sr[c]);
+  #pragma unroll
+        for (int c = 8; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+                         a.scale_log2;
+        // lazy rescale: move the reference max only when the block max exceeds it by more than 8
+        float alpha = 1.f;
+        if (mx > m + 8.f || (m == -INFINITY && mx != -INFINITY)) {
+          alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - mx);
+          m = mx;
+        }
+        const float m_use = (m == -INFINITY) ? 0.f : m;
+        // P = 2^(scale s - m) as bf16 pairs over the first 64 columns of S: keys 0-63 first (P columns
+        // 0-31), released to the P V MMA at once, then keys 64-127. Blocks that no row of the warp
+        // masks may take part of the exponentials on the FMA pipe (exp2_poly_pair); masked entries
+        // always go through ex2, which returns exactly 0 for them.
+        const bool poly_ok = kPolyEighths > 0 && !__any_sync(0xffffffffu, kbase + kBN - 1 > row_limit);
+        const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), nm2 = f2_pack(-m_use, -m_use);
+        uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};  // four packed sum chains
+  #pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t pk[32];
+  #pragma unroll
+          for (int c = 64 * hf; c < 64 * hf + 64; c += 2) {
+            float x0, x1, p0, p1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2), x0, x1);
+            if (((c >> 1) & 7) < kPolyEighths && poly_ok) {
+              exp2_poly_pair(x0, x1, p0, p1);
+            } else {
+              p0 = fast_exp2(x0);
+              p1 = fast_exp2(x1);
+            }
+            rs2[(c >> 1) & 3] = f2_add(rs2[(c >> 1) & 3], f2_pack(p0, p1));
+            pk[(c - 64 * hf) / 2] = pack_bf16(p0, p1);
+          }
+          tmem_st16(tS + 32 * hf, pk);
+          tmem_st16(tS + 32 * hf + 16, pk + 16);
+          // S of block j is complete, hence so is P V of block j - 1: O may be rescaled now, before
+          // the first P V of block j is released.
+          if (hf == 0 && j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+  #pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 16) {
+              uint32_t orr[16];
+              tmem_ld16(tO + c0, orr);
+              tmem_wait_ld();
+  #pragma unroll
+              for (int e = 0; e < 16; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+              tmem_st16(tO + c0, orr);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(p_full + 2 * t + hf);
+        }
+        float rsum[8];
+  #pragma unroll
+        for (int u = 0; u < 4; ++u) f2_unpack(rs2[u], rsum[2 * u], rsum[2 * u + 1]);
+        l = l * alpha + (((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) + ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7])));
       }
+      sb += n_kv;
+      // epilogue: O / l -> bf16, lse = (m + log2 l) ln 2. O leaves TMEM in two 64-column halves;
+      // once both are in registers the next item's first P V may overwrite it.
+      const bool have = ok && n_kv > 0;
+      if (have) ok = wait_warp(o_done + t, ct & 1);
       tc_fence_after();
-      const int kbase = j * kBN;
-      // the whole 128-column row of S in registers: one round trip to TMEM
-      uint32_t sr[kBN];
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const bool store = qrow < a.Sq;
+      uint16_t* orow = a.o + ((static_cast<long long>(b) * a.Sq + qrow) * a.Hq + h) * D;
+      uint32_t orr[D];
+      if (have && ok) {
 #pragma unroll
-      for (int c = 0; c < kBN; c += 16) tmem_ld16(tS + c, sr + c);
-      tmem_wait_ld();
-      if (kbase + kBN - 1 > row_limit) {  // the block crosses this row's last visible key
-#pragma unroll
-        for (int c = 0; c < kBN; ++c)
-          if (kbase + c > row_limit) sr[c] = __float_as_uint(-INFINITY);
-      }
-      float mx8[8];  // eight independent max chains
-#pragma unroll
-      for (int c = 0; c < 8; ++c) mx8[c] = __uint_as_float(sr[c]);
-#pragma unroll
-      for (int c = 8; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
-                       a.scale_log2;
-      // lazy rescale: move the reference max only when the block max exceeds it by more than 8
-      float alpha = 1.f;
-      if (mx > m + 8.f || (m == -INFINITY && mx != -INFINITY)) {
-        alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - mx);
-        m = mx;
-      }
-      const float m_use = (m == -INFINITY) ? 0.f : m;
-      // P = 2^(scale s - m) as bf16 pairs over the first 64 columns of S: keys 0-63 first (P columns
-      // 0-31), released to the P V MMA at once, then keys 64-127. Blocks that no row of the warp
-      // masks may take part of the exponentials on the FMA pipe (exp2_poly_pair); masked entries
-      // always go through ex2, which returns exactly 0 for them.
-      const bool poly_ok = kPolyEighths > 0 && !__any_sync(0xffffffffu, kbase + kBN - 1 > row_limit);
-      const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), nm2 = f2_pack(-m_use, -m_use);
-      uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};  // four packed sum chains
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 64 * hf; c < 64 * hf + 64; c += 2) {
-          float x0, x1, p0, p1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2), x0, x1);
-          if (((c >> 1) & 7) < kPolyEighths && poly_ok) {
-            exp2_poly_pair(x0, x1, p0, p1);
-          } else {
-            p0 = fast_exp2(x0);
-            p1 = fast_exp2(x1);
-          }
-          rs2[(c >> 1) & 3] = f2_add(rs2[(c >> 1) & 3], f2_pack(p0, p1));
-          pk[(c - 64 * hf) / 2] = pack_bf16(p0, p1);
-        }
-        tmem_st16(tS + 32 * hf, pk);
-        tmem_st16(tS + 32 * hf + 16, pk + 16);
-        // S of block j is complete, hence so is P V of block j - 1: O may be rescaled now, before
-        // the first P V of block j is released.
-        if (hf == 0 && j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 16) {
-            uint32_t orr[16];
-            tmem_ld16(tO + c0, orr);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-            tmem_st16(tO + c0, orr);
-          }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(p_full + 2 * t + hf);
-      }
-      float rsum[8];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) f2_unpack(rs2[u], rsum[2 * u], rsum[2 * u + 1]);
-      l = l * alpha + (((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) + ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7])));
-    }
-    if (ok && n_kv > 0) ok = wait_warp(o_done + t, 0);
-    tc_fence_after();
-    // epilogue: O / l -> bf16, lse = (m + log2 l) ln 2
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    const bool store = qrow < a.Sq;
-    uint16_t* orow = a.o + ((static_cast<long long>(b) * a.Sq + qrow) * a.Hq + h) * D;
-#pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 16) {
-      uint32_t orr[16];
-      if (ok && n_kv > 0) {
-        tmem_ld16(tO + c0, orr);
+        for (int c0 = 0; c0 < D; c0 += 16) tmem_ld16(tO + c0, orr + c0);
         tmem_wait_ld();
       } else {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) orr[e] = 0u;
+        for (int e = 0; e < D; ++e) orr[e] = 0u;
+      }
+      if (n_kv > 0) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(o_free + t);
+        ++ct;
       }
       if (store) {
-        uint4 w0, w1;
-        w0.x = pack_bf16(__uint_as_float(orr[0]) * inv, __uint_as_float(orr[1]) * inv);
-        w0.y = pack_bf16(__uint_as_float(orr[2]) * inv, __uint_as_float(orr[3]) * inv);
-        w0.z = pack_bf16(__uint_as_float(orr[4]) * inv, __uint_as_float(orr[5]) * inv);
-        w0.w = pack_bf16(__uint_as_float(orr[6]) * inv, __uint_as_float(orr[7]) * inv);
-        w1.x = pack_bf16(__uint_as_float(orr[8]) * inv, __uint_as_float(orr[9]) * inv);
-        w1.y = pack_bf16(__uint_as_float(orr[10]) * inv, __uint_as_float(orr[11]) * inv);
-        w1.z = pack_bf16(__uint_as_float(orr[12]) * inv, __uint_as_float(orr[13]) * inv);
-        w1.w = pack_bf16(__uint_as_float(orr[14]) * inv, __uint_as_float(orr[15]) * inv);
-        *reinterpret_cast<uint4*>(orow + c0) = w0;
-        *reinterpret_cast<uint4*>(orow + c0 + 8) = w1;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 16) {
+          uint4 w0, w1;
+          w0.x = pack_bf16(__uint_as_float(orr[c0 + 0]) * inv, __uint_as_float(orr[c0 + 1]) * inv);
+          w0.y = pack_bf16(__uint_as_float(orr[c0 + 2]) * inv, __uint_as_float(orr[c0 + 3]) * inv);
+          w0.z = pack_bf16(__uint_as_float(orr[c0 + 4]) * inv, __uint_as_float(orr[c0 + 5]) * inv);
+          w0.w = pack_bf16(__uint_as_float(orr[c0 + 6]) * inv, __uint_as_float(orr[c0 + 7]) * inv);
+          w1.x = pack_bf16(__uint_as_float(orr[c0 + 8]) * inv, __uint_as_float(orr[c0 + 9]) * inv);
+          w1.y = pack_bf16(__uint_as_float(orr[c0 + 10]) * inv, __uint_as_float(orr[c0 + 11]) * inv);
+          w1.z = pack_bf16(__uint_as_float(orr[c0 + 12]) * inv, __uint_as_float(orr[c0 + 13]) * inv);
+          w1.w = pack_bf16(__uint_as_float(orr[c0 + 14]) * inv, __uint_as_float(orr[c0 + 15]) * inv);
+          *reinterpret_cast<uint4*>(orow + c0) = w0;
+          *reinterpret_cast<uint4*>(orow + c0 + 8) = w1;
+        }
+        a.lse[(static_cast<long long>(b) * a.Hq + h) * a.Sq + qrow] =
+            l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
       }
     }
-    if (store) a.lse[(static_cast<long long>(b) * a.Hq + h) * a.Sq + qrow] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
   }
 
   tc_fence_before();
@@ -446,7 +535,14 @@ cudaError_t launch_fwd_sm100_d(const Problem& p, const void* q, const void* k, c
   a.o = static_cast<uint16_t*>(o);
   a.lse = lse;
   a.status = device_status_ptr();
-  dim3 grid(p.Hq * p.B, a.n_pairs);
+  // a persistent grid: one CTA per SM, each walking its share of the (head, tile pair) items
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const long long n_items = static_cast<long long>(p.Hq) * p.B * a.n_pairs;
+  dim3 grid(static_cast<unsigned>(std::min<long long>(n_items, sms)));
   {
     LaunchScope ls("fwd_sm100", st);
     fwd_sm100_kernel<D><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);

@@ -48,30 +48,36 @@
 namespace attn {
 namespace {
 
-constexpr int kBM = 128;   // query rows per iteration
+constexpr int kBM = 64;    // query rows per tile (two tiles in flight)
 constexpr int kBN = 128;   // keys per CTA
-constexpr int kThreads = 320;
-constexpr int kAtom = 128 * 128;  // a 128-row x 128-byte swizzle atom (16 KB)
+constexpr int kThreads = 448;       // 14 warps
+constexpr int kAtom = 128 * 128;    // a 128-row x 128-byte swizzle atom (16 KB)
+constexpr int kAtom64 = 64 * 128;   // a 64-row x 128-byte swizzle atom (8 KB)
 
 template <int D>
 struct BwdCfg {
   static constexpr int kAtoms = D / 64;
-  static constexpr int kTileBytes = kAtoms * kAtom;  // 128 rows x D bf16
-  static constexpr int kStages = 2;
+  static constexpr int kKVBytes = kAtoms * kAtom;    // 128 key rows x D bf16 (K, V)
+  static constexpr int kQBytes = kAtoms * kAtom64;   // 64 query rows x D bf16 (Q, dO)
+  static constexpr int kStages = 4;                  // Q / dO ring: two tiles in flight + two ahead
   static constexpr int kOffK = 0;
-  static constexpr int kOffV = kOffK + kTileBytes;
-  static constexpr int kOffQ = kOffV + kTileBytes;
-  static constexpr int kOffDO = kOffQ + kStages * kTileBytes;
-  static constexpr int kOffDS = kOffDO + kStages * kTileBytes;  // 128 keys x 128 rows bf16 = 2 atoms
+  static constexpr int kOffV = kOffK + kKVBytes;
+  static constexpr int kOffQ = kOffV + kKVBytes;
+  static constexpr int kOffDO = kOffQ + kStages * kQBytes;
+  static constexpr int kOffDS = kOffDO + kStages * kQBytes;  // [2 tiles] 128 keys x 64 queries bf16
   static constexpr int kOffBar = kOffDS + 2 * kAtom;
-  static constexpr int kNumBars = 1 + 2 * kStages + 9;
+  static constexpr int kNumBars = 1 + 2 * kStages + 6 * 2 + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  // lse2 and Delta of the current tile, read as float4: 16-byte aligned whatever the barrier count
+  // lse2 and Delta of each group's current tile ([2 groups][lse2 64, Delta 64]), read as float4
   static constexpr int kOffRow = (kOffMisc + 64 + 15) & ~15;
-  static constexpr int kSmemBytes = kOffRow + 2 * kBM * 4 + 1024;
+  static constexpr int kSmemBytes = kOffRow + 2 * 2 * kBM * 4 + 1024;
   static_assert(kOffRow % 16 == 0, "the lse2 / Delta rows are read with 16-byte loads");
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-  static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
+  // TMEM: tile buffer b holds S^T / P^T / dQ^T at 128 b and dP^T / dS^T at 128 b + 64 (64 columns
+  // each); dV at 256, dK at 384
+  __host__ __device__ static constexpr uint32_t colS(int b) { return 128u * b; }
+  __host__ __device__ static constexpr uint32_t colDP(int b) { return 128u * b + 64u; }
+  static constexpr uint32_t kColDV = 256, kColDK = 384;
 };
 
 struct BwdArgs {
@@ -115,23 +121,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sV = smem + C::kOffV;
   uint8_t* sQ = smem + C::kOffQ;
   uint8_t* sDO = smem + C::kOffDO;
-  uint8_t* sDS = smem + C::kOffDS;
+  uint8_t* sDS = smem + C::kOffDS;  // [tile buffer] 128 keys x 64 queries, one 128-byte swizzle atom
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* kv_full = bars;
-  uint64_t* q_full = bars + 1;
-  uint64_t* q_empty = q_full + C::kStages;
-  uint64_t* s_full = q_empty + C::kStages;  // S^T of a tile is in TMEM
-  uint64_t* dp_full = s_full + 1;           // dP^T of a tile is in TMEM
-  uint64_t* p_full = dp_full + 1;           // P^T, dS^T written (TMEM and shared)
-  uint64_t* ds_free = p_full + 1;           // dQ^T MMA done reading dS^T in shared memory
-  uint64_t* dq_full = ds_free + 1;          // dQ^T of a tile is in TMEM
-  uint64_t* dq_free = dq_full + 1;          // the drain has read dQ^T out of TMEM
-  uint64_t* all_done = dq_free + 1;
+  uint64_t* q_full = bars + 1;               // [stage]
+  uint64_t* q_empty = q_full + C::kStages;   // [stage]
+  uint64_t* s_full = q_empty + C::kStages;   // [buffer] S^T of a tile is in TMEM
+  uint64_t* dp_full = s_full + 2;            // [buffer] dP^T of a tile is in TMEM
+  uint64_t* p_full = dp_full + 2;            // [buffer] P^T and dS^T written (TMEM and shared)
+  uint64_t* ds_free = p_full + 2;            // [buffer] the dQ^T MMA has read dS^T in shared memory
+  uint64_t* dq_full = ds_free + 2;           // [buffer] dQ^T of a tile is in TMEM
+  uint64_t* dq_free = dq_full + 2;           // [buffer] the drain has read dQ^T out of TMEM
+  uint64_t* all_done = dq_free + 2;
   uint64_t* drain = all_done + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
-  float* sLse = reinterpret_cast<float*>(smem + C::kOffRow);  // [kBM]
-  float* sDlt = sLse + kBM;                                    // [kBM]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = static_cast<int>(blockIdx.x) % a.Hkv;
@@ -146,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     qt0 = qmin <= 0 ? 0 : qmin / kBM;
   }
   const int n_q = qt0 < n_qt_all ? n_qt_all - qt0 : 0;
-  const int n_it = G * n_q;
+  const int n_it = G * n_q;  // tiles: query head (slow) x query tile (fast)
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -154,22 +158,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(q_full + s, 1);
       mbar_init(q_empty + s, 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(dp_full, 1);
-    mbar_init(p_full, 4);
-    mbar_init(ds_free, 1);
-    mbar_init(dq_full, 1);
-    mbar_init(dq_free, 4);
+    for (int bb = 0; bb < 2; ++bb) {
+      mbar_init(s_full + bb, 1);
+      mbar_init(dp_full + bb, 1);
+      mbar_init(p_full + bb, 4);
+      mbar_init(ds_free + bb, 1);
+      mbar_init(dq_full + bb, 1);
+      mbar_init(dq_free + bb, 4);
+    }
     mbar_init(all_done, 1);
     mbar_init(drain, 1);
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == 12 && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -180,11 +186,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0 && n_it > 0) {
-      constexpr uint32_t kTx = kBN * D * 2;
-      mbar_arrive_expect_tx(kv_full, 2 * kTx);
+      constexpr uint32_t kTxKV = kBN * D * 2, kTxQ = kBM * D * 2;
+      mbar_arrive_expect_tx(kv_full, 2 * kTxKV);
 #pragma unroll
       for (int at = 0; at < C::kAtoms; ++at) {
         tma_load_4d(sK + at * kAtom, &tmK, kv_full, at * 64, g, k0, b);
@@ -196,11 +202,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int h = g * G + j / n_q;
         const int qt = qt0 + j % n_q;
         if (!mbar_wait(q_empty + s, ((j / C::kStages) & 1) ^ 1, abort, a.status)) break;
-        mbar_arrive_expect_tx(q_full + s, 2 * kTx);
+        mbar_arrive_expect_tx(q_full + s, 2 * kTxQ);
 #pragma unroll
         for (int at = 0; at < C::kAtoms; ++at) {
-          tma_load_4d(sQ + s * C::kTileBytes + at * kAtom, &tmQ, q_full + s, at * 64, h, qt * kBM, b);
-          tma_load_4d(sDO + s * C::kTileBytes + at * kAtom, &tmDO, q_full + s, at * 64, h, qt * kBM, b);
+          tma_load_4d(sQ + s * C::kQBytes + at * kAtom64, &tmQ, q_full + s, at * 64, h, qt * kBM, b);
+          tma_load_4d(sDO + s * C::kQBytes + at * kAtom64, &tmDO, q_full + s, at * 64, h, qt * kBM, b);
         }
         issued = j + 1;
       }
@@ -208,10 +214,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = max(0, issued - C::kStages); j < issued; ++j)
         wait_drain(q_full + j % C::kStages, (j / C::kStages) & 1);
     }
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ------------------------------------------------------------------ MMA issuer
     if (n_it > 0) {  // the whole warp runs the loop; one elected lane issues each MMA
-      constexpr uint32_t kIdS = idesc_bf16_f32(kBN, kBM, 0, 0);  // S^T, dP^T
+      constexpr uint32_t kIdS = idesc_bf16_f32(kBN, kBM, 0, 0);  // S^T, dP^T: M 128 keys, N 64 queries
       constexpr uint32_t kIdG = idesc_bf16_f32(kBN, D, 0, 1);    // dV, dK (A in TMEM)
       constexpr uint32_t kIdQ = idesc_bf16_f32(128, kBM, 1, 1);  // dQ^T (M = 128 also for D = 64)
       // base descriptors, built once; each MMA only moves the start address
@@ -219,75 +225,66 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t kV = sdesc_sw128(smem_u32(sV), 16, 1024);
       const uint64_t kQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t kDO = sdesc_sw128(smem_u32(sDO), 16, 1024);
-      const uint64_t mQ = sdesc_sw128(smem_u32(sQ), kAtom, 1024);    // MN-major operands
-      const uint64_t mDO = sdesc_sw128(smem_u32(sDO), kAtom, 1024);
+      const uint64_t mQ = sdesc_sw128(smem_u32(sQ), kAtom64, 1024);  // MN-major operands
+      const uint64_t mDO = sdesc_sw128(smem_u32(sDO), kAtom64, 1024);
       const uint64_t mK = sdesc_sw128(smem_u32(sK), kAtom, 1024);
       const uint64_t mDS = sdesc_sw128(smem_u32(sDS), kAtom, 1024);
       auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
         return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, a.status)) != 0;
       };
-      // S^T (into the S^T columns) and dP^T (into the dP^T columns) of tile jt
-      auto issue_s = [&](int jt) {
-        const uint64_t q = sdesc_advance(kQ, (jt % C::kStages) * C::kTileBytes);
+      // S^T = K Q^T (or dP^T = V dO^T) of tile jt into its buffer: K = D in steps of 16; the 128-row
+      // A tile and the 64-row B tile have different atom strides
+      auto issue_scores = [&](int jt, uint64_t aK, uint64_t bQ, uint32_t col, uint64_t* bar) {
+        const uint64_t bq = sdesc_advance(bQ, (jt % C::kStages) * C::kQBytes);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
-          umma_ss_warp(tmem + C::kColS, sdesc_advance(kK, off), sdesc_advance(q, off), kIdS, kk > 0);
-        }
-        umma_commit_warp(s_full);
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ss_warp(tmem + col, sdesc_advance(aK, (kk >> 2) * kAtom + (kk & 3) * 32),
+                       sdesc_advance(bq, (kk >> 2) * kAtom64 + (kk & 3) * 32), kIdS, kk > 0);
+        umma_commit_warp(bar);
       };
-      auto issue_dp = [&](int jt) {
-        const uint64_t dO = sdesc_advance(kDO, (jt % C::kStages) * C::kTileBytes);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
-          umma_ss_warp(tmem + C::kColDP, sdesc_advance(kV, off), sdesc_advance(dO, off), kIdS, kk > 0);
+      bool ok = wait(kv_full, 0);
+      for (int jt = 0; ok && jt < min(2, n_it); ++jt) {
+        if (!wait(q_full + jt % C::kStages, (jt / C::kStages) & 1)) {
+          ok = false;
+          break;
         }
-        umma_commit_warp(dp_full);
-      };
-      bool ok = wait(kv_full, 0) && wait(q_full, 0);
-      if (ok) {
         tc_fence_after();
-        issue_s(0);
-        issue_dp(0);
+        issue_scores(jt, kK, kQ, C::colS(jt & 1), s_full + (jt & 1));
+        issue_scores(jt, kV, kDO, C::colDP(jt & 1), dp_full + (jt & 1));
       }
       for (int j = 0; ok && j < n_it; ++j) {
-        const int s = j % C::kStages;
-        const bool more = j + 1 < n_it;
-        // gradients of tile j once P^T and dS^T are written
-        if (!wait(p_full, j & 1)) break;
+        const int bb = j & 1, s = j % C::kStages;
+        // gradients of tile j once its P^T and dS^T are written
+        if (!wait(p_full + bb, (j >> 1) & 1)) break;
         tc_fence_after();
-        const uint64_t q = sdesc_advance(mQ, s * C::kTileBytes), dO = sdesc_advance(mDO, s * C::kTileBytes);
-        // dV += P^T dO: K = 128 query rows in 8 steps of 16 (8 TMEM columns each)
+        const uint64_t q = sdesc_advance(mQ, s * C::kQBytes), dO = sdesc_advance(mDO, s * C::kQBytes);
+        // dV += P^T dO and dK += dS^T Q: K = 64 query rows in 4 steps of 16 (8 TMEM columns each)
 #pragma unroll
         for (int kk = 0; kk < kBM / 16; ++kk)
-          umma_ts_warp(tmem + C::kColDV, tmem + C::kColS + kk * 8, sdesc_advance(dO, kk * 16 * 128), kIdG,
+          umma_ts_warp(tmem + C::kColDV, tmem + C::colS(bb) + kk * 8, sdesc_advance(dO, kk * 16 * 128), kIdG,
                        (j > 0 || kk > 0));
-        // S^T of tile j + 1 over P^T of tile j, which dV has just read: the next tile's P^T can be
-        // computed while dK and dQ^T of this tile run
-        if (more) {
-          if (!wait(q_full + (j + 1) % C::kStages, ((j + 1) / C::kStages) & 1)) break;
-          tc_fence_after();
-          issue_s(j + 1);
-        }
-        // dK += dS^T Q
 #pragma unroll
         for (int kk = 0; kk < kBM / 16; ++kk)
-          umma_ts_warp(tmem + C::kColDK, tmem + C::kColDP + kk * 8, sdesc_advance(q, kk * 16 * 128), kIdG,
+          umma_ts_warp(tmem + C::kColDK, tmem + C::colDP(bb) + kk * 8, sdesc_advance(q, kk * 16 * 128), kIdG,
                        (j > 0 || kk > 0));
-        // dQ^T = K^T dS^T over the dP^T / dS^T columns (dK has read dS^T): K = 128 keys, 8 steps of 16
+        // dQ^T = K^T dS^T over the tile's S^T / P^T columns (dV has read P^T): K = 128 keys in 8 steps
+        const uint64_t ds = sdesc_advance(mDS, bb * kAtom);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_ss_warp(tmem + C::kColDP, sdesc_advance(mK, kk * 16 * 128), sdesc_advance(mDS, kk * 16 * 128), kIdQ,
+          umma_ss_warp(tmem + C::colS(bb), sdesc_advance(mK, kk * 16 * 128), sdesc_advance(ds, kk * 16 * 128), kIdQ,
                        kk > 0);
         umma_commit_warp(q_empty + s);
-        umma_commit_warp(ds_free);
-        umma_commit_warp(dq_full);
-        // dP^T of tile j + 1 over dQ^T of tile j: the drain must have read it
-        if (more) {
-          if (!wait(dq_free, j & 1)) break;
+        umma_commit_warp(ds_free + bb);
+        umma_commit_warp(dq_full + bb);
+        if (j + 2 < n_it) {
+          // tile j + 2 in the same buffer: dP^T at once (dK has read dS^T), S^T once the drain has
+          // read dQ^T
+          if (!wait(q_full + (j + 2) % C::kStages, ((j + 2) / C::kStages) & 1)) break;
           tc_fence_after();
-          issue_dp(j + 1);
+          issue_scores(j + 2, kV, kDO, C::colDP(bb), dp_full + bb);
+          if (!wait(dq_free + bb, (j >> 1) & 1)) break;
+          tc_fence_after();
+          issue_scores(j + 2, kK, kQ, C::colS(bb), s_full + bb);
         }
       }
       umma_commit_warp(all_done);
@@ -295,19 +292,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_drain(drain, 0);
       __syncwarp();
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------------ score warps (row = key)
+    // Group gg = warp / 4 scores the tiles j with j % 2 == gg (tile buffer gg); its four warps
+    // cover the four TMEM lane quarters, one key row per thread, 64 query columns.
     griddep_wait();  // lse2 and Delta come from bwd_prep
-    const int t = threadIdx.x;  // TMEM lane == key row in the tile
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_addr + C::kColS, tDP = tmem + lane_addr + C::kColDP;
+    const int gg = warp >> 2;
+    const int t = threadIdx.x & 127;  // TMEM lane == key row in the tile
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_addr + C::colS(gg), tDP = tmem + lane_addr + C::colDP(gg);
+    uint8_t* sDSg = sDS + gg * kAtom;
+    float* sLse = reinterpret_cast<float*>(smem + C::kOffRow) + gg * 2 * kBM;  // [64]
+    float* sDlt = sLse + kBM;                                                  // [64]
     const int key = k0 + t;
     bool ok = true;
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
       const bool r = mbar_wait(bar, parity, abort, a.status);
       return __all_sync(0xffffffffu, r);
     };
-    for (int j = 0; j < n_it; ++j) {
+    for (int j = gg; j < n_it; j += 2) {
       const int h = g * G + j / n_q;
       const int q0 = (qt0 + j % n_q) * kBM;
       const float* lse2 = a.lse2 + (static_cast<long long>(b) * a.Hq + h) * a.Sq_pad + q0;
@@ -318,159 +321,153 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int cmin = a.causal ? key - (a.Sk - a.Sq) - q0 : 0;
       const int cmax = key < a.Sk ? kBM : 0;
       const bool unmasked = __all_sync(0xffffffffu, cmin <= 0 && cmax == kBM) != 0;
-      // this tile's lse2 and Delta into shared memory, once every score warp is done with the last
-      // tile's; the loads overlap the wait for S^T. Every score warp runs all n_it iterations (one
-      // whose wait failed only passes the barriers), so the named barriers always complete.
-      named_barrier(1, 128);
+      // this tile's lse2 and Delta into the group's shared rows, once its four warps are done with
+      // the last tile's; every warp of the group runs all its tiles (one whose wait failed only
+      // passes the barriers), so the named barriers always complete
+      named_barrier(1 + gg, 128);
       if (ok) {
-        sLse[t] = lse2[t];
-        sDlt[t] = dlt[t];
+        if (t < kBM) sLse[t] = lse2[t];
+        else sDlt[t - kBM] = dlt[t - kBM];
       }
-      named_barrier(1, 128);
+      named_barrier(1 + gg, 128);
       if (!ok) continue;
-      if (!wait_warp(s_full, j & 1)) {
+      if (!wait_warp(s_full + gg, (j >> 1) & 1)) {
         ok = false;
         continue;
       }
       tc_fence_after();
-      // P^T = 2^(S^T scale log2e - lse2) in two halves of 64 query columns, as bf16 pairs over the
-      // first 64 S^T columns (already read), where the dV MMA and the dS^T step below read them
+      // P^T = 2^(S^T scale log2e - lse2), as bf16 pairs over the first 32 columns (already read):
+      // the dV MMA reads them there; this thread keeps its own for dS^T
+      uint32_t pk[kBM / 2];
+      {
+        uint32_t sr[kBM];
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t sr[64], pk[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 16) tmem_ld16(tS + hf * 64 + c, sr + c);
+        for (int c = 0; c < kBM; c += 16) tmem_ld16(tS + c, sr + c);
         tmem_wait_ld();
 #pragma unroll
-        for (int c4 = 0; c4 < 64; c4 += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(sLse + hf * 64 + c4);  // same for every lane
+        for (int c4 = 0; c4 < kBM; c4 += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(sLse + c4);  // same for every lane
           const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
           for (int e = 0; e < 4; e += 2) {
-            const int c = hf * 64 + c4 + e;
-            float p0 = fast_exp2(fmaf(__uint_as_float(sr[c4 + e]), a.scale_log2, -lv[e]));
-            float p1 = fast_exp2(fmaf(__uint_as_float(sr[c4 + e + 1]), a.scale_log2, -lv[e + 1]));
+            const int c = c4 + e;
+            float p0 = fast_exp2(fmaf(__uint_as_float(sr[c]), a.scale_log2, -lv[e]));
+            float p1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), a.scale_log2, -lv[e + 1]));
             if (!unmasked) {
               p0 = (c >= cmin && c < cmax) ? p0 : 0.f;
               p1 = (c + 1 >= cmin && c + 1 < cmax) ? p1 : 0.f;
             }
-            pk[(c4 + e) / 2] = pack_bf16(p0, p1);
+            pk[c / 2] = pack_bf16(p0, p1);
           }
         }
-        tmem_st16(tS + hf * 32, pk);
-        tmem_st16(tS + hf * 32 + 16, pk + 16);
+        tmem_st16(tS, pk);
+        tmem_st16(tS + 16, pk + 16);
       }
-      if (!wait_warp(dp_full, j & 1)) {
+      if (!wait_warp(dp_full + gg, (j >> 1) & 1)) {
         ok = false;
         continue;
       }
-      // shared dS^T of the previous tile must have been consumed by its dQ^T MMA
-      if (!wait_warp(ds_free, (j & 1) ^ 1)) {
+      // the shared dS^T of tile j - 2 must have been consumed by its dQ^T MMA
+      if (!wait_warp(ds_free + gg, ((j >> 1) & 1) ^ 1)) {
         ok = false;
         continue;
       }
-      tmem_wait_st();  // this thread's P^T stores are visible to its own loads below
       tc_fence_after();
-      // dS^T = P^T (dP^T - Delta), from the bf16 P^T above, in two halves of 64 query columns
+      // dS^T = P^T (dP^T - Delta) in two halves of 32 query columns
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
-        uint32_t dp[64], pk[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 16) tmem_ld16(tDP + hf * 64 + c, dp + c);
-        tmem_ld16(tS + hf * 32, pk);
-        tmem_ld16(tS + hf * 32 + 16, pk + 16);
+        uint32_t dp[32];
+        tmem_ld16(tDP + hf * 32, dp);
+        tmem_ld16(tDP + hf * 32 + 16, dp + 16);
         tmem_wait_ld();
-        uint32_t dk[32];
+        uint32_t dk[16];
 #pragma unroll
-        for (int c4 = 0; c4 < 64; c4 += 4) {
-          const float4 d4 = *reinterpret_cast<const float4*>(sDlt + hf * 64 + c4);
+        for (int c4 = 0; c4 < 32; c4 += 4) {
+          const float4 d4 = *reinterpret_cast<const float4*>(sDlt + hf * 32 + c4);
           const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
           for (int e = 0; e < 4; e += 2) {
-            const uint32_t pw = pk[(c4 + e) / 2];
+            const uint32_t pw = pk[(hf * 32 + c4 + e) / 2];
             const float d0 = bf16_lo(pw) * (__uint_as_float(dp[c4 + e]) - dv4[e]);
             const float d1 = bf16_hi(pw) * (__uint_as_float(dp[c4 + e + 1]) - dv4[e + 1]);
             dk[(c4 + e) / 2] = pack_bf16(d0, d1);
           }
         }
-        // dS^T over dP^T columns 32 hf .. 32 hf + 31 (already read), and to shared memory: key row
-        // t, query columns 64 hf .. 64 hf + 63 = swizzle atom hf
-        tmem_st16(tDP + hf * 32, dk);
-        tmem_st16(tDP + hf * 32 + 16, dk + 16);
+        // dS^T over dP^T columns 16 hf .. 16 hf + 15 (already read), and to shared memory: key row
+        // t, query columns 32 hf .. 32 hf + 31 = 16-byte chunks 4 hf .. 4 hf + 3 of the atom
+        tmem_st16(tDP + hf * 16, dk);
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          *reinterpret_cast<uint4*>(sDS + hf * kAtom + sw128_offset(t, u)) =
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<uint4*>(sDSg + sw128_offset(t, hf * 4 + u)) =
               make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
       }
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(p_full + gg);
     }
-    // dK / dV epilogue: TMEM rows -> bf16 global rows of this key tile
+    // dK / dV epilogue: TMEM rows -> bf16 global rows of this key tile (group 0: dV, group 1: dK)
     if (ok && n_it > 0) ok = wait_warp(all_done, 0);
     tc_fence_after();
     const bool store = key < a.Sk;
     const long long row = ((static_cast<long long>(b) * a.Sk + key) * a.Hkv + g) * D;
+    const uint32_t col = gg == 0 ? C::kColDV : C::kColDK;
+    const float mul = gg == 0 ? 1.f : a.scale;
+    uint16_t* dst = (gg == 0 ? a.dv : a.dk) + row;
 #pragma unroll 1
-    for (int which = 0; which < 2; ++which) {
-      const uint32_t col = which == 0 ? C::kColDV : C::kColDK;
-      const float mul = which == 0 ? 1.f : a.scale;
-      uint16_t* dst = (which == 0 ? a.dv : a.dk) + row;
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 16) {
-        uint32_t r[16];
-        if (ok && n_it > 0) {
-          tmem_ld16(tmem + lane_addr + col + c0, r);
-          tmem_wait_ld();
-        } else {
+    for (int c0 = 0; c0 < D; c0 += 16) {
+      uint32_t r[16];
+      if (ok && n_it > 0) {
+        tmem_ld16(tmem + lane_addr + col + c0, r);
+        tmem_wait_ld();
+      } else {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) r[e] = 0u;
-        }
-        if (store) {
-          uint4 w0, w1;
-          w0.x = pack_bf16(__uint_as_float(r[0]) * mul, __uint_as_float(r[1]) * mul);
-          w0.y = pack_bf16(__uint_as_float(r[2]) * mul, __uint_as_float(r[3]) * mul);
-          w0.z = pack_bf16(__uint_as_float(r[4]) * mul, __uint_as_float(r[5]) * mul);
-          w0.w = pack_bf16(__uint_as_float(r[6]) * mul, __uint_as_float(r[7]) * mul);
-          w1.x = pack_bf16(__uint_as_float(r[8]) * mul, __uint_as_float(r[9]) * mul);
-          w1.y = pack_bf16(__uint_as_float(r[10]) * mul, __uint_as_float(r[11]) * mul);
-          w1.z = pack_bf16(__uint_as_float(r[12]) * mul, __uint_as_float(r[13]) * mul);
-          w1.w = pack_bf16(__uint_as_float(r[14]) * mul, __uint_as_float(r[15]) * mul);
-          *reinterpret_cast<uint4*>(dst + c0) = w0;
-          *reinterpret_cast<uint4*>(dst + c0 + 8) = w1;
-        }
+        for (int e = 0; e < 16; ++e) r[e] = 0u;
+      }
+      if (store) {
+        uint4 w0, w1;
+        w0.x = pack_bf16(__uint_as_float(r[0]) * mul, __uint_as_float(r[1]) * mul);
+        w0.y = pack_bf16(__uint_as_float(r[2]) * mul, __uint_as_float(r[3]) * mul);
+        w0.z = pack_bf16(__uint_as_float(r[4]) * mul, __uint_as_float(r[5]) * mul);
+        w0.w = pack_bf16(__uint_as_float(r[6]) * mul, __uint_as_float(r[7]) * mul);
+        w1.x = pack_bf16(__uint_as_float(r[8]) * mul, __uint_as_float(r[9]) * mul);
+        w1.y = pack_bf16(__uint_as_float(r[10]) * mul, __uint_as_float(r[11]) * mul);
+        w1.z = pack_bf16(__uint_as_float(r[12]) * mul, __uint_as_float(r[13]) * mul);
+        w1.w = pack_bf16(__uint_as_float(r[14]) * mul, __uint_as_float(r[15]) * mul);
+        *reinterpret_cast<uint4*>(dst + c0) = w0;
+        *reinterpret_cast<uint4*>(dst + c0 + 8) = w1;
       }
     }
   } else {
-    // ------------------------------------------------------------------ dQ drain (warps 4-7)
-    griddep_wait();  // bwd_prep has cleared the accumulator
+    // ------------------------------------------------------------------ dQ drain (warps 8-11)
     // Thread e holds TMEM lane e = head-dim column d of dQ^T; for each group of four query rows the
     // warp's 32 lanes add 32 consecutive columns x 4 rows (512 contiguous bytes) into the
     // interleaved accumulator.
-    const int wq = warp - 4;
+    griddep_wait();  // bwd_prep has cleared the accumulator
+    const int wq = warp - 8;
     const int d = wq * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tQ = tmem + lane_addr + C::kColDP;
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
       const bool r = mbar_wait(bar, parity, abort, a.status);
       return __all_sync(0xffffffffu, r);
     };
     for (int j = 0; j < n_it; ++j) {
+      const int bb = j & 1;
       const int h = g * G + j / n_q;
       const int q0 = (qt0 + j % n_q) * kBM;
-      if (!wait_warp(dq_full, j & 1)) break;
+      if (!wait_warp(dq_full + bb, (j >> 1) & 1)) break;
       tc_fence_after();
-      // the whole dQ^T row of this lane in one round trip; then its columns may be reused at once
+      // the whole dQ^T row of this lane (64 query columns) in one round trip; then its columns may
+      // be reused at once
       uint32_t r[kBM];
 #pragma unroll
-      for (int c = 0; c < kBM; c += 16) tmem_ld16(tQ + c, r + c);
+      for (int c = 0; c < kBM; c += 16) tmem_ld16(tmem + lane_addr + C::colS(bb) + c, r + c);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(dq_free);
-      if (d < D) {  // at D = 64 warps 6 and 7 hold no dQ column
+      if (lane == 0) mbar_arrive(dq_free + bb);
+      if (d < D) {  // at D = 64 warps 10 and 11 hold no dQ column
         // rows q0 + 4i .. q0 + 4i + 3 of column d: 16 contiguous bytes at acc + 4 D i
         float* acc = a.dq_acc + ((static_cast<long long>(b) * a.Hq + h) * a.Sq_pad + q0) * D + 4 * d;
 #pragma unroll
@@ -481,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

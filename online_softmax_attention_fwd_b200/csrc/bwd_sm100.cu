@@ -10,33 +10,35 @@
 //   bwd_prep        Delta_i = dO_i . O_i, lse in base 2, and the fp32 dQ accumulator cleared, all
 //                   padded to a multiple of 128 query rows (padding rows: lse2 = +inf, Delta = 0);
 //   bwd_sm100       one CTA per (128-key tile, kv head): loops over the group's query heads x
-//                   128-row query tiles, keeps dK and dV for its keys in TMEM, and adds each tile's
+//                   64-row query tiles, keeps dK and dV for its keys in TMEM, and adds each tile's
 //                   dQ into the fp32 accumulator;
 //   bwd_dq_convert  dQ = scale * accumulator, rounded to bf16.
 //
 // The main kernel works on transposed score tiles so that keys sit on the TMEM lanes:
-//   S^T = K Q^T and dP^T = V dO^T            (M = 128 keys, N = 128 query rows, K = D).
-// One thread per key computes P^T = 2^(S^T scale log2e - lse2) as soon as S^T is in TMEM, and
-// dS^T = P^T (dP^T - Delta) once dP^T is; each is written back as bf16 over the first 64 columns of
-// its own TMEM tile, and dS^T also goes to shared memory (128-byte swizzle). Then
+//   S^T = K Q^T and dP^T = V dO^T            (M = 128 keys, N = 64 query rows, K = D).
+// Two query tiles are in flight: tile j lives in TMEM buffer j % 2 (S^T / P^T in 64 columns, dP^T /
+// dS^T / dQ^T in 64 more) and is scored by warpgroup j % 2. One thread per key computes
+// P^T = 2^(S^T scale log2e - lse2) as soon as S^T is in TMEM (kept in registers and written back as
+// bf16 over the first 32 S^T columns), and dS^T = P^T (dP^T - Delta) once dP^T is (written back over
+// the first 32 dP^T columns and into the tile's dS^T tile in shared memory, 128-byte swizzle). Then
 //   dV += P^T dO,  dK += dS^T Q              (A = P^T / dS^T in TMEM, B = dO / Q MN-major in SMEM)
-//   dQ^T = K^T dS^T                          (M = D, N = 128 query rows, K = 128 keys; both in SMEM)
-// with S^T of the next tile issued right after dV (over P^T, which dV has read), so the next tile's
-// P^T is computed while dK and dQ^T of this tile run; dQ^T goes over the dP^T columns once dK has
-// read dS^T, and the next dP^T waits until the drain has read dQ^T. MMAs execute in issue order,
-// which is what makes each overwrite in TMEM safe. dQ is produced transposed (head dim on the TMEM
-// lanes, query rows on the columns), and the fp32 accumulator interleaves groups of four query
-// rows, [B, Hq, Sq_pad / 4, D, 4], so that a lane adds four consecutive rows of its column with one
-// 16-byte vector reduction and a warp instruction covers 512 contiguous bytes. For D = 64 the dQ^T MMA still runs with M = 128; the upper 64
-// TMEM lanes hold values that are never read.
-// TMEM columns: S^T / P^T [0,128), dP^T / dS^T / dQ^T [128,256), dV [256,256+D), dK [384,384+D).
+//   dQ^T = K^T dS^T                          (M = D, N = 64 query rows, K = 128 keys; both in SMEM)
+// Issue order for tile j: dV, then S^T of tile j + 2 over P^T (which dV has read), so the group
+// computes the next P^T while dK, dQ^T and the drain of this tile run; dK, then dQ^T over the dP^T
+// columns (which dK has read); dP^T of tile j + 2 once the drain has read dQ^T. MMAs execute in
+// issue order, which is what makes each overwrite in TMEM safe. dQ is produced transposed (head
+// dim on the TMEM lanes, query rows on the columns), and the fp32 accumulator interleaves groups of
+// four query rows, [B, Hq, Sq_pad / 4, D, 4], so that a lane adds four consecutive rows of its
+// column with one 16-byte vector reduction and a warp instruction covers 512 contiguous bytes. For
+// D = 64 the dQ^T MMA still runs with M = 128; the upper 64 TMEM lanes hold values that are never
+// read. TMEM columns: buffer b at [128 b, 128 b + 128), dV [256, 256 + D), dK [384, 384 + D).
 //
-// Warp roles (320 threads): warps 0-3 scores (one key row per thread; at the end the dK/dV
-// epilogue), warps 4-7 dQ drain (one TMEM lane = one head-dim column per thread: the whole dQ^T
-// row in one tcgen05.ld, TMEM released at once, then 4-wide fp32 vector reductions into the
-// interleaved accumulator),
-// warp 8 TMA producer (K, V once; Q and dO tiles through a 2-stage ring), warp 9 TMEM allocator
-// and MMA issuer (one elected lane of a converged warp). Every wait is bounded.
+// Warp roles (448 threads): warps 0-3 / 4-7 score the even / odd tiles (one key row per thread; at
+// the end group 0 stores dV and group 1 dK), warps 8-11 dQ drain (one TMEM lane = one head-dim
+// column per thread: the whole dQ^T row in one tcgen05.ld, TMEM released at once, then 4-wide fp32
+// vector reductions into the interleaved accumulator), warp 12 TMA producer (K, V once; Q and dO
+// tiles through a 4-stage ring), warp 13 TMEM allocator and MMA issuer (one elected lane of a
+// converged warp). Every wait is bounded.
 #include <math.h>
 
 #include <algorithm>
@@ -73,7 +75,7 @@ struct BwdCfg {
   static constexpr int kSmemBytes = kOffRow + 2 * 2 * kBM * 4 + 1024;
   static_assert(kOffRow % 16 == 0, "the lse2 / Delta rows are read with 16-byte loads");
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-  // TMEM: tile buffer b holds S^T / P^T / dQ^T at 128 b and dP^T / dS^T at 128 b + 64 (64 columns
+  // TMEM: tile buffer b holds S^T / P^T at 128 b and dP^T / dS^T / dQ^T at 128 b + 64 (64 columns
   // each); dV at 256, dK at 384
   __host__ __device__ static constexpr uint32_t colS(int b) { return 128u * b; }
   __host__ __device__ static constexpr uint32_t colDP(int b) { return 128u * b + 64u; }
@@ -263,28 +265,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < kBM / 16; ++kk)
           umma_ts_warp(tmem + C::kColDV, tmem + C::colS(bb) + kk * 8, sdesc_advance(dO, kk * 16 * 128), kIdG,
                        (j > 0 || kk > 0));
+        // S^T of tile j + 2 (same buffer) over P^T of tile j, which dV has just read: the group
+        // computes the next P^T while dK, dQ^T and the drain of this tile run
+        if (j + 2 < n_it) {
+          if (!wait(q_full + (j + 2) % C::kStages, ((j + 2) / C::kStages) & 1)) break;
+          tc_fence_after();
+          issue_scores(j + 2, kK, kQ, C::colS(bb), s_full + bb);
+        }
 #pragma unroll
         for (int kk = 0; kk < kBM / 16; ++kk)
           umma_ts_warp(tmem + C::kColDK, tmem + C::colDP(bb) + kk * 8, sdesc_advance(q, kk * 16 * 128), kIdG,
                        (j > 0 || kk > 0));
-        // dQ^T = K^T dS^T over the tile's S^T / P^T columns (dV has read P^T): K = 128 keys in 8 steps
+        // dQ^T = K^T dS^T over the tile's dP^T / dS^T columns (dK has read dS^T): K = 128 keys in 8 steps
         const uint64_t ds = sdesc_advance(mDS, bb * kAtom);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_ss_warp(tmem + C::colS(bb), sdesc_advance(mK, kk * 16 * 128), sdesc_advance(ds, kk * 16 * 128), kIdQ,
+          umma_ss_warp(tmem + C::colDP(bb), sdesc_advance(mK, kk * 16 * 128), sdesc_advance(ds, kk * 16 * 128), kIdQ,
                        kk > 0);
         umma_commit_warp(q_empty + s);
         umma_commit_warp(ds_free + bb);
         umma_commit_warp(dq_full + bb);
         if (j + 2 < n_it) {
-          // tile j + 2 in the same buffer: dP^T at once (dK has read dS^T), S^T once the drain has
-          // read dQ^T
-          if (!wait(q_full + (j + 2) % C::kStages, ((j + 2) / C::kStages) & 1)) break;
-          tc_fence_after();
-          issue_scores(j + 2, kV, kDO, C::colDP(bb), dp_full + bb);
+          // dP^T of tile j + 2 over dQ^T of tile j, once the drain has read it
           if (!wait(dq_free + bb, (j >> 1) & 1)) break;
           tc_fence_after();
-          issue_scores(j + 2, kK, kQ, C::colS(bb), s_full + bb);
+          issue_scores(j + 2, kV, kDO, C::colDP(bb), dp_full + bb);
         }
       }
       umma_commit_warp(all_done);
@@ -462,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // be reused at once
       uint32_t r[kBM];
 #pragma unroll
-      for (int c = 0; c < kBM; c += 16) tmem_ld16(tmem + lane_addr + C::colS(bb) + c, r + c);
+      for (int c = 0; c < kBM; c += 16) tmem_ld16(tmem + lane_addr + C::colDP(bb) + c, r + c);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();

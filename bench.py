@@ -487,12 +487,18 @@ def run_ours(args):
 
 def run_case(name):
     """One launch of each kernel of a workload and nothing else (a small command for ncu captures):
-    `prefill` = the 4k GQA causal forward and backward, `decode` = the 48-stream split-KV decode."""
+    `prefill` = the 4k GQA causal forward and backward, `decode` = the 48-stream split-KV decode,
+    `long` = the forward of the long-prefill workload at S = 16384 (the 44k workload's construction
+    and kernel at a size that a full ncu capture handles; about 0.4 GB on the device)."""
     import torch
     import online_softmax_attention_fwd_b200 as attn
     from online_softmax_attention_fwd_b200 import workloads as W
     dev = torch.device("cuda")
-    if name == "prefill":
+    if name == "long":
+        w = W.long_prefill_44k(S=16384)
+        q, k, v = (t.to(dev) for t in (w.q, w.k, w.v))
+        attn.fwd(q, k, v, causal=True, scale=w.scale)
+    elif name == "prefill":
         w = W.gqa_prefill_4k("A")
         q, k, v, do = (t.to(dev) for t in (w.q, w.k, w.v, w.do))
         o, lse = attn.fwd(q, k, v, causal=True, scale=w.scale)
@@ -515,7 +521,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true")
-    ap.add_argument("--case", choices=["prefill", "decode"],
+    ap.add_argument("--case", choices=["prefill", "decode", "long"],
                     help="run one launch of each kernel of this workload and exit (for profilers)")
     args = ap.parse_args()
     if args.case:

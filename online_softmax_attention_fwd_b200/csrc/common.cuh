@@ -59,25 +59,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// 2^x on the FMA and integer pipes, for x <= 128 (results below 2^-126 are returned as 0), so that
-// part of a softmax's exponentials can bypass the transcendental unit. Written from the
-// decomposition 2^x = 2^n * 2^f with n = round(x) and f = x - n in [-1/2, 1/2]: adding 1.5 * 2^23
-// rounds x to an integer held in the low mantissa bits; 2^f comes from a cubic fitted to 2^f on
-// [-1/2, 1/2] (weighted least squares on the relative error at Chebyshev nodes, maximum relative
-// error 7.7e-5, well under bf16's 2^-8); n is then added to the exponent field.
-__device__ __forceinline__ float exp2_poly(float x) {
-  const float kRound = 12582912.f;  // 1.5 * 2^23
-  const float xc = fmaxf(x, -126.f);
-  const float r = xc + kRound;
-  const float n = r - kRound;
-  const float f = xc - n;
-  float p = fmaf(0.05508868380751114f, f, 0.24260405145947936f);
-  p = fmaf(p, f, 0.6932762416819607f);
-  p = fmaf(p, f, 0.9999289403695112f);
-  const float y = __int_as_float(__float_as_int(p) + (__float_as_int(r) << 23));
-  return x < -126.f ? 0.f : y;
-}
-
 // Packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction updates two values held in a 64-bit
 // register pair.
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
@@ -102,27 +83,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
-}
-
-// 2^x for a pair of finite x, with the pair arithmetic on the FMA pipe (the polynomial of exp2_poly
-// above, two values per instruction). Inputs are clamped at -126, so an input below -126 gives a
-// value near 2^-126 rather than 0: callers use it only where such a value is negligible against the
-// sum it joins (never for masked entries, which must be exactly 0).
-__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
-  const float kRound = 12582912.f;  // 1.5 * 2^23
-  const uint64_t xc = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
-  const uint64_t r = f2_add(xc, f2_pack(kRound, kRound));     // round(x) in the low mantissa bits
-  const uint64_t n = f2_add(r, f2_pack(-kRound, -kRound));    // round(x) as a float
-  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), xc);      // x - round(x) in [-1/2, 1/2]
-  uint64_t p = f2_fma(f, f2_pack(0.05508868380751114f, 0.05508868380751114f),
-                      f2_pack(0.24260405145947936f, 0.24260405145947936f));
-  p = f2_fma(p, f, f2_pack(0.6932762416819607f, 0.6932762416819607f));
-  p = f2_fma(p, f, f2_pack(0.9999289403695112f, 0.9999289403695112f));
-  float p0, p1, r0, r1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(r, r0, r1);
-  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(r0) << 23));
-  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(r1) << 23));
 }
 
 // Warp-level tensor-core fragments (m16n8k16, bf16 inputs, fp32 accumulators), for contractions

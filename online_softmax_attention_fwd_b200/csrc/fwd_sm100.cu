@@ -50,12 +50,6 @@ namespace {
 constexpr int kBM = 128;   // query rows per tile (two tiles per CTA)
 constexpr int kBN = 128;   // keys per block
 constexpr int kThreads = 320;
-// Eighths of each unmasked block's exponentials computed on the FMA pipe instead of ex2 (the
-// transcendental unit is the softmax's bottleneck).
-#ifndef ATTN_FWD_POLY_EIGHTHS
-#define ATTN_FWD_POLY_EIGHTHS 0
-#endif
-constexpr int kPolyEighths = ATTN_FWD_POLY_EIGHTHS;
 constexpr int kAtom = 128 * 128;  // 128 rows x 128 bytes (16 KB)
 
 template <int D>
@@ -410,10 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float m_use = (m == -INFINITY) ? 0.f : m;
         // P = 2^(scale s - m) as bf16 pairs over the first 64 columns of S: keys 0-63 first (P columns
-        // 0-31), released to the P V MMA at once, then keys 64-127. Blocks that no row of the warp
-        // masks may take part of the exponentials on the FMA pipe (exp2_poly_pair); masked entries
-        // always go through ex2, which returns exactly 0 for them.
-        const bool poly_ok = kPolyEighths > 0 && !__any_sync(0xffffffffu, kbase + kBN - 1 > row_limit);
+        // 0-31), released to the P V MMA at once, then keys 64-127 (ex2 of a masked -inf is 0)
         const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), nm2 = f2_pack(-m_use, -m_use);
         uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};  // four packed sum chains
   #pragma unroll
@@ -423,12 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 64 * hf; c < 64 * hf + 64; c += 2) {
             float x0, x1, p0, p1;
             f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2), x0, x1);
-            if (((c >> 1) & 7) < kPolyEighths && poly_ok) {
-              exp2_poly_pair(x0, x1, p0, p1);
-            } else {
-              p0 = fast_exp2(x0);
-              p1 = fast_exp2(x1);
-            }
+            p0 = fast_exp2(x0);
+            p1 = fast_exp2(x1);
             rs2[(c >> 1) & 3] = f2_add(rs2[(c >> 1) & 3], f2_pack(p0, p1));
             pk[(c - 64 * hf) / 2] = pack_bf16(p0, p1);
           }

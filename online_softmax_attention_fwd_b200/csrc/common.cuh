@@ -59,6 +59,14 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// max of three floats in one instruction (three-input max.f32, sm_100); exact, so the order in which
+// a row maximum is formed does not change it.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction updates two values held in a 64-bit
 // register pair.
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {

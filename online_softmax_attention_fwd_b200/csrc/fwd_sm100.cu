@@ -9,9 +9,13 @@
 // The two contractions are dense, so they run as tcgen05.mma with fp32 accumulators in tensor
 // memory; the row statistics run on the CUDA cores, one thread per row.
 //
-// The grid is persistent (one CTA per SM). A work item is two 128-row query tiles of one head, and
-// the CTA streams each 128-key K/V block once for both. Items are sorted longest first (under a
-// causal mask the last tile pairs see the most keys) and dealt to the CTAs in snake order. Across
+// The grid is persistent (one CTA per SM). A work item is two 128-row query tiles that read the
+// same keys, and the CTA streams each 128-key K/V block once for both. When each key/value head
+// serves an even number of query heads, the two tiles are the same rows of two query heads of one
+// group: under a causal mask both then see the same number of blocks, and items come in 128-row
+// steps of length. Otherwise they are two consecutive row tiles of one head. Items are sorted
+// longest first (under a causal mask the last rows see the most keys) and dealt to the CTAs in
+// snake order. Across
 // items the K/V ring runs on without a pause. The next item's Q is loaded as soon as the current
 // item's last S is complete, and a tile's epilogue overlaps the next item's first S; the first P V
 // of an item waits only until that epilogue has read O out of TMEM (barrier o_free).
@@ -74,7 +78,12 @@ struct FwdArgs {
   int B, Hq, Hkv, Sq, Sk;
   int causal;
   float scale_log2;  // softmax scale * log2(e)
-  int n_pairs;       // pairs of 128-row query tiles
+  // A work item is two 128-row query tiles that read the same K/V blocks. With head_pairs, the two
+  // tiles are the same rows of query heads 2 hs and 2 hs + 1 (one key/value group, as the head
+  // count ratio is even); otherwise they are rows 256 s .. 256 s + 255 of one head.
+  int head_pairs;
+  int n_slots;       // row positions per head set: 128-row tiles (head_pairs) or 256-row pairs
+  int n_hsets;       // head sets per batch entry: Hq / 2 (head_pairs) or Hq
   uint16_t* o;
   float* lse;
   int* status;
@@ -130,17 +139,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BH = a.B * a.Hq;
-  const int n_items = BH * a.n_pairs;
+  const int BH = a.B * a.n_hsets;
+  const int n_items = BH * a.n_slots;
   const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
-  // item i: tile pair n_pairs - 1 - i / BH (the longest pairs first under a causal mask), (b, h) = i % BH
+  // item i: row position n_slots - 1 - i / BH (the longest items first under a causal mask) of head
+  // set i % BH; tile t covers head h + t dh, rows q0 + t dq
+  const int dh = a.head_pairs ? 1 : 0, dq = a.head_pairs ? 0 : kBM;
   auto item_of = [&](int i, int& b, int& h, int& q0, int& n0, int& n1) {
-    const int bh = i % BH, pair = a.n_pairs - 1 - i / BH;
-    b = bh / a.Hq;
-    h = bh % a.Hq;
-    q0 = pair * 2 * kBM;
+    const int bh = i % BH, slot = a.n_slots - 1 - i / BH;
+    b = bh / a.n_hsets;
+    h = (bh % a.n_hsets) * (a.head_pairs ? 2 : 1);
+    q0 = slot * (a.head_pairs ? kBM : 2 * kBM);
     n0 = tile_blocks(a, q0);
-    n1 = tile_blocks(a, q0 + kBM);
+    n1 = tile_blocks(a, q0 + dq);
   };
 
   if (threadIdx.x == 0) {
@@ -202,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if ((t == 0 ? n0 : n1) == 0) continue;
 #pragma unroll
           for (int at = 0; at < C::kAtoms; ++at)
-            tma_load_4d(sQ + t * C::kTileBytes + at * kAtom, &tmQ, q_full, at * 64, h, q0 + t * kBM, b);
+            tma_load_4d(sQ + t * C::kTileBytes + at * kAtom, &tmQ, q_full, at * 64, h + t * dh, q0 + t * dq, b);
         }
         ++qk;
         for (int j = 0; j < nmax; ++j) {
@@ -367,7 +378,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int b, h, q0, n0, n1;
       item_of(i, b, h, q0, n0, n1);
       const int n_kv = t == 0 ? n0 : n1;
-      const int qrow = q0 + t * kBM + row;
+      h += t * dh;
+      const int qrow = q0 + t * dq + row;
       int row_limit = a.Sk - 1;  // largest visible key index for this row
       if (a.causal) row_limit = min(row_limit, qrow + a.Sk - a.Sq);
       float m = -INFINITY, l = 0.f;
@@ -388,13 +400,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kBN; ++c)
             if (kbase + c > row_limit) sr[c] = __float_as_uint(-INFINITY);
         }
-        float mx8[8];  // eight independent max chains
+        float mx8[8];  // eight independent max chains, two new columns per three-input max
   #pragma unroll
-        for (int c = 0; c < 8; ++c) mx8[c] = __uint_as_float(sr[c]);
+        for (int c = 0; c < 8; ++c) mx8[c] = fmaxf(__uint_as_float(sr[c]), __uint_as_float(sr[c + 8]));
   #pragma unroll
-        for (int c = 8; c < kBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+        for (int c = 16; c < kBN; c += 16)
+  #pragma unroll
+          for (int u = 0; u < 8; ++u)
+            mx8[u] = fmax3(mx8[u], __uint_as_float(sr[c + u]), __uint_as_float(sr[c + 8 + u]));
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                               fmaxf(mx8[6], mx8[7])) *
                          a.scale_log2;
         // lazy rescale: move the reference max only when the block max exceeds it by more than 8
         float alpha = 1.f;
@@ -518,7 +533,9 @@ cudaError_t launch_fwd_sm100_d(const Problem& p, const void* q, const void* k, c
   a.Sk = p.Sk;
   a.causal = p.causal;
   a.scale_log2 = p.scale * kLog2e;
-  a.n_pairs = (p.Sq + 2 * kBM - 1) / (2 * kBM);
+  a.head_pairs = (p.Hq / p.Hkv) % 2 == 0 ? 1 : 0;
+  a.n_slots = a.head_pairs ? (p.Sq + kBM - 1) / kBM : (p.Sq + 2 * kBM - 1) / (2 * kBM);
+  a.n_hsets = a.head_pairs ? p.Hq / 2 : p.Hq;
   a.o = static_cast<uint16_t*>(o);
   a.lse = lse;
   a.status = device_status_ptr();
@@ -528,7 +545,7 @@ cudaError_t launch_fwd_sm100_d(const Problem& p, const void* q, const void* k, c
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  const long long n_items = static_cast<long long>(p.Hq) * p.B * a.n_pairs;
+  const long long n_items = static_cast<long long>(a.n_hsets) * p.B * a.n_slots;
   dim3 grid(static_cast<unsigned>(std::min<long long>(n_items, sms)));
   {
     LaunchScope ls("fwd_sm100", st);

@@ -255,8 +255,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t dQ0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
     const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);
     const uint64_t dV0 = sdesc_sw128(smem_u32(sV), kAtom, 1024);
+    // polling waits: the issuer reacts to a completed P or K/V phase without a wake-up delay
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, a.status)) != 0;
+      return __all_sync(0xffffffffu, mbar_wait_spin(bar, parity, abort, a.status)) != 0;
     };
     long long kvb = 0;      // ring position of the item's first K/V block
     long long k_ready = -1, v_ready = -1;  // last K / V block this warp has waited for

@@ -396,6 +396,14 @@ def run_ours(args):
                 "fwd_ms": tf * 1e3, "fwd_tflops": fb / tf / 1e12, "bwd_ms": tb * 1e3,
                 "bwd_tflops": 2.5 * fb / tb / 1e12}
             del qb, kb, vb, dob, ob, lb
+        # the same 48 decode streams read from a paged cache (64-key pages, shuffled pool)
+        pc = W.paged_from_packed(dec, 64, seed=0)
+        kp, vp, bt, sl = (t.to(dev) for t in (pc.k_pages, pc.v_pages, pc.block_table, pc.seq_lens))
+        t_pg = time_part(lambda: attn.decode_paged(qd, kp, vp, bt, sl, max_splits=16, scale=dec.scale, out=od,
+                                                   lse=lsed, workspace=wsd), iters)
+        components["decode48_paged64"] = {"ms": t_pg * 1e3, "kv_gbs": b_dec / t_pg / 1e9,
+                                          "frac_of_hbm": b_dec / t_pg / 1e9 / peaks["hbm_gbs"]}
+        del kp, vp, bt, sl, pc
         w5 = W.long_prefill_44k()
         q5, k5, v5 = (t.to(dev) for t in (w5.q, w5.k, w5.v))
         o5, l5 = attn.fwd(q5, k5, v5, causal=True, scale=w5.scale)

@@ -155,6 +155,28 @@ attn_status_t attn_decode_splitkv_static(const void* q, const void* k, const voi
 /* Host helper: the built-in split count for a stream of L keys (the rule named above). */
 int attn_decode_default_splits(int L, int max_splits);
 
+/* Split-KV decode over a paged key/value cache (the pages have no counterpart: a serving engine
+ * keeps its decode streams' caches in fixed-size pages of one pool, and this entry point reads
+ * them in place, with the same split + combine and the same monoid as attn_decode_splitkv).
+ *
+ *   k_pages, v_pages [num_pages, page_size, Hkv, D] bf16: the pools. Key t of stream n is row
+ *   t % page_size of page block_table[n * max_pages + t / page_size].
+ *   block_table [N, max_pages] int32 DEVICE array of page ids; seq_lens [N] int32 DEVICE array of
+ *   stream lengths (L_n is clamped to [0, max_pages * page_size]). Only the entries for pages that
+ *   hold keys of a stream are read. A page id outside [0, num_pages) is not read: its keys count as
+ *   zeros and the device status records ATTN_ERR_INVALID_ARG (read it with attn_get_device_status).
+ *   page_size: a multiple of 16, at least 16; num_pages * page_size < 2^31.
+ *   Rows of a stream's last page past its length may hold anything (also NaN): they are not read.
+ *   Chunks are whole 16-key blocks (ceil(L_n / C_n) rounded up to 16), so for the same split count
+ *   the partial triples can differ from attn_decode_splitkv's by rounding only.
+ *   q, o, lse, num_splits, max_splits, scale, workspace: as for attn_decode_splitkv (the same
+ *   workspace size, attn_decode_workspace_size(N, Hq, D, max_splits)). D is 64 or 128. */
+attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                                const int* block_table, int max_pages, const int* seq_lens, int page_size,
+                                int num_pages, const int* num_splits, int max_splits, void* o, float* lse,
+                                int N, int Hq, int Hkv, int D, float scale, void* workspace,
+                                size_t workspace_bytes, attn_stream_t stream);
+
 /* ------------------------------------------------------------------------------------------ *
  * Status and introspection.
  * ------------------------------------------------------------------------------------------ */
@@ -163,7 +185,8 @@ int attn_decode_default_splits(int L, int max_splits);
 const char* attn_status_string(attn_status_t status);
 
 /* Waits for `stream`, then reads and clears the library's device status word on the current
- * device: ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel gave up a bounded wait since the last read. */
+ * device: ATTN_OK, ATTN_ERR_TIMEOUT if a kernel gave up a bounded wait since the last read, or
+ * ATTN_ERR_INVALID_ARG if attn_decode_paged met a page id outside its pool. */
 attn_status_t attn_get_device_status(attn_stream_t stream);
 
 /* Number of CUDA kernels this library has launched in this process (all devices, all calls). */

@@ -6,7 +6,7 @@ Scaled-dot-product attention computed as one reduction under the online-softmax 
 * ``fwd`` -- bf16 prefill forward (tcgen05 tensor cores, TMA, TMEM), GQA, causal, lse output;
 * ``bwd`` -- bf16 backward to dQ, dK, dV;
 * ``decode`` -- split-KV decode over packed varlen caches, partial (m, l, o) triples merged by the
-  monoid in a combine kernel;
+  monoid in a combine kernel; ``decode_paged`` -- the same over a paged cache (block table);
 * ``fwd_f32`` / ``bwd_f32`` -- genuine fp32 CUDA-core versions.
 
 The C entry points are declared in ``include/attn.h``; this package only marshals torch tensors to
@@ -20,6 +20,7 @@ from ._binding import (  # noqa: F401
     bwd_f32,
     bwd_workspace_size,
     decode,
+    decode_paged,
     decode_workspace_size,
     default_splits,
     device_status,

@@ -32,6 +32,9 @@ SIGNATURES = [
     ("attn_decode_splitkv", _I, [_P] * 5 + [_I] + [_P, _P] + [_I] * 4 + [_F, _P, _S, _P]),
     ("attn_decode_splitkv_static", _I, [_P] * 5 + [_I] + [_P, _P] + [_I] * 4 + [_F, _P]),
     ("attn_decode_default_splits", _I, [_I, _I]),
+    # q, k_pages, v_pages, block_table, max_pages, seq_lens, page_size, num_pages, num_splits,
+    # max_splits, o, lse, N, Hq, Hkv, D, scale, workspace, workspace_bytes, stream
+    ("attn_decode_paged", _I, [_P] * 4 + [_I, _P, _I, _I, _P, _I, _P, _P] + [_I] * 4 + [_F, _P, _S, _P]),
     ("attn_status_string", ctypes.c_char_p, [_I]),
     ("attn_get_device_status", _I, [_P]),
     ("attn_launch_count", ctypes.c_uint64, []),
@@ -188,6 +191,39 @@ def decode(q, k, v, kv_offsets, num_splits=None, max_splits: int = 16, scale: Op
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
     _check("attn_decode_splitkv", lib().attn_decode_splitkv(
         _ptr(q), _ptr(k), _ptr(v), _ptr(kv_offsets), _ptr(num_splits), int(max_splits), _ptr(o),
+        _ptr(lse) if want_lse else None, N, Hq, Hkv, D, scale, _ptr(workspace), workspace.numel(), _stream()))
+    return o, (lse if want_lse else None)
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seq_lens, num_splits=None, max_splits: int = 16,
+                 scale: Optional[float] = None, want_lse: bool = True, out=None, lse=None, workspace=None):
+    """Split-KV decode over a paged cache via attn_decode_paged: returns (O [N,Hq,D] bf16, lse or None).
+
+    k_pages, v_pages [num_pages, page_size, Hkv, D] bf16; block_table [N, max_pages] int32 page ids;
+    seq_lens [N] int32. Key t of stream n is k_pages[block_table[n, t // page_size], t % page_size].
+    """
+    _expect(q, "q", torch.bfloat16, 3)
+    _expect(k_pages, "k_pages", torch.bfloat16, 4)
+    _expect(v_pages, "v_pages", torch.bfloat16, 4)
+    _expect(block_table, "block_table", torch.int32, 2)
+    _expect(seq_lens, "seq_lens", torch.int32, 1)
+    if num_splits is not None:
+        _expect(num_splits, "num_splits", torch.int32, 1)
+    N, Hq, D = q.shape
+    num_pages, page_size, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    if (tuple(v_pages.shape) != tuple(k_pages.shape) or k_pages.shape[3] != D or block_table.shape[0] != N
+            or seq_lens.numel() != N):
+        raise ValueError("shape mismatch in paged decode arguments")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    if want_lse and lse is None:
+        lse = torch.empty((N, Hq), dtype=torch.float32, device=q.device)
+    need = decode_workspace_size(N, Hq, D, max_splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check("attn_decode_paged", lib().attn_decode_paged(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), int(block_table.shape[1]), _ptr(seq_lens),
+        int(page_size), int(num_pages), _ptr(num_splits), int(max_splits), _ptr(o),
         _ptr(lse) if want_lse else None, N, Hq, Hkv, D, scale, _ptr(workspace), workspace.numel(), _stream()))
     return o, (lse if want_lse else None)
 

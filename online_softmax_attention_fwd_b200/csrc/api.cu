@@ -250,7 +250,38 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v, c
   const DecodeProblem p{N, Hq, Hkv, D, max_splits, scale};
   const cudaError_t e = launch_decode(p, q, k, v, kv_offsets, num_splits, o, lse, workspace,
                                       static_cast<cudaStream_t>(stream));
-  if (e == cudaSuccess) g_last_path[2] = "decode_splitkv_simt";
+  if (e == cudaSuccess) g_last_path[2] = "decode_splitkv_mma16816";
+  return launch_status(e);
+}
+
+attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int* block_table,
+                                int max_pages, const int* seq_lens, int page_size, int num_pages,
+                                const int* num_splits, int max_splits, void* o, float* lse, int N, int Hq, int Hkv,
+                                int D, float scale, void* workspace, size_t workspace_bytes,
+                                attn_stream_t stream) {
+  if (N <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (max_splits < 1 || max_splits > 64) return ATTN_ERR_INVALID_ARG;
+  if (N > 65535 || static_cast<long long>(N) * Hq >= (1ll << 31)) return ATTN_ERR_INVALID_ARG;
+  if (page_size < 16 || page_size % 16 != 0 || num_pages <= 0 || max_pages <= 0) return ATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(num_pages) * page_size >= (1ll << 31) ||
+      static_cast<long long>(max_pages) * page_size >= (1ll << 31) ||
+      static_cast<long long>(N) * max_pages >= (1ll << 40))
+    return ATTN_ERR_INVALID_ARG;
+  attn_status_t s = check_ptrs(q, k_pages, v_pages, block_table, o);
+  if (s != ATTN_OK) return s;
+  if (!seq_lens) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(seq_lens)) return ATTN_ERR_ALIGNMENT;
+  if (num_splits && !aligned16(num_splits)) return ATTN_ERR_ALIGNMENT;
+  if (lse && !aligned16(lse)) return ATTN_ERR_ALIGNMENT;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < decode_workspace_bytes(N, Hq, D, max_splits)) return ATTN_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_ALIGNMENT;
+  if (!device_is_sm100()) return ATTN_ERR_UNSUPPORTED;
+  const DecodeProblem p{N, Hq, Hkv, D, max_splits, scale};
+  const cudaError_t e =
+      launch_decode_paged(p, q, k_pages, v_pages, block_table, max_pages, seq_lens, page_size, num_pages, num_splits,
+                          o, lse, workspace, static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess) g_last_path[2] = "decode_splitkv_paged_mma16816";
   return launch_status(e);
 }
 

@@ -15,6 +15,7 @@ namespace attn {
 
 // Status codes written into the device status word (same values as attn_status_t).
 constexpr int kStatusOk = 0;
+constexpr int kStatusBadArg = 1;    // an index read on the device is out of range (ATTN_ERR_INVALID_ARG)
 constexpr int kStatusTimeout = 6;
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer (2 s): far above any

@@ -24,6 +24,11 @@
 // tensor maps carry a nominal row extent and the kernel issues a 16-row box only when the whole box
 // lies below T; the cache's last partial block is fetched in 16-byte pieces with bulk copies. No
 // copy ever touches memory past the caller's K and V buffers.
+// A paged cache (pages of a multiple of 16 keys, a block table per stream) runs through the same
+// kernels: chunks are then whole 16-key blocks, so a block lies in one page and its box starts at
+// the page's pool row; the stream's last partial block is copied row by row and the rest of it
+// zero-filled, since the rest of a page may hold anything. A page id outside the pool is not read:
+// its rows count as zeros and the device status records ATTN_ERR_INVALID_ARG.
 #include <math.h>
 
 #include <algorithm>
@@ -58,6 +63,27 @@ __device__ __forceinline__ int stream_splits(const int* num_splits, int n, int L
     return c < 1 ? 1 : (c > max_splits ? max_splits : c);
   }
   return decode_split_rule(L, max_splits);
+}
+
+// Where the keys of each stream live. Contiguous: stream n owns rows offsets[n] .. offsets[n+1] - 1
+// of the packed caches. Paged (block_table != null): key t of stream n is row t % page_size of page
+// block_table[n * max_pages + t / page_size] of a pool of num_pages pages, and the stream has
+// seq_lens[n] keys (clamped to [0, max_pages * page_size]).
+struct DecKV {
+  const int* offsets;
+  const int* seq_lens;
+  const int* block_table;
+  int max_pages, page_size, num_pages;
+};
+
+__device__ __forceinline__ void dec_stream(const DecKV& kv, int n, int& start, int& L) {
+  if (kv.block_table) {
+    start = 0;
+    L = min(max(kv.seq_lens[n], 0), kv.max_pages * kv.page_size);
+  } else {
+    start = kv.offsets[n];
+    L = kv.offsets[n + 1] - start;
+  }
 }
 
 constexpr int kDecBlk = 16;              // keys per block (two lanes per key while scoring)
@@ -100,11 +126,14 @@ struct DecItem {
 // Item slot idx -> item; false for slots past the stream's split count. Slots are ordered chunk
 // index slowest, so the first chunks of every stream and kv head come first.
 // The item whose fields are (n, c, gi) -> it; L = the stream's length, C_n its split count.
+// With `aligned`, chunks are rounded up to whole 16-key blocks (a paged cache: a block must not
+// straddle two pages); the last chunks of a stream may then be empty.
 template <int GT>
 __device__ __forceinline__ void dec_item_fill(int n, int c, int gi, int start, int L, int C_n, int Hq, int Hkv,
-                                              DecItem& it) {
+                                              bool aligned, DecItem& it) {
   const int G = Hq / Hkv, npass = G / GT;
-  const int chunk = (L + C_n - 1) / C_n;
+  int chunk = (L + C_n - 1) / C_n;
+  if (aligned) chunk = (chunk + kDecBlk - 1) / kDecBlk * kDecBlk;
   it.n = n;
   it.c = c;
   it.g = gi / npass;
@@ -120,7 +149,7 @@ __device__ __forceinline__ void dec_item_fill(int n, int c, int gi, int start, i
 // kv heads of one chunk are consecutive items, so neighbouring CTAs read the same cache rows at
 // about the same time (a row holds every kv head's keys side by side).
 template <int GT>
-__device__ __forceinline__ void dec_item_dense(int k, int N, int Hq, int Hkv, const int* offsets, const int* base,
+__device__ __forceinline__ void dec_item_dense(int k, int N, int Hq, int Hkv, const DecKV& kv, const int* base,
                                                DecItem& it) {
   int lo = 0, hi = N;  // largest n with base[n] <= k
   while (hi - lo > 1) {
@@ -130,23 +159,24 @@ __device__ __forceinline__ void dec_item_dense(int k, int N, int Hq, int Hkv, co
   const int NG = Hkv * ((Hq / Hkv) / GT);
   const int C_n = (base[lo + 1] - base[lo]) / NG;
   const int r = k - base[lo];
-  const int start = offsets[lo];
-  dec_item_fill<GT>(lo, r / NG, r % NG, start, offsets[lo + 1] - start, C_n, Hq, Hkv, it);
+  int start, L;
+  dec_stream(kv, lo, start, L);
+  dec_item_fill<GT>(lo, r / NG, r % NG, start, L, C_n, Hq, Hkv, kv.block_table != nullptr, it);
 }
 
 template <int GT>
-__device__ __forceinline__ bool dec_item(long long idx, int N, int Hq, int Hkv, const int* offsets,
+__device__ __forceinline__ bool dec_item(long long idx, int N, int Hq, int Hkv, const DecKV& kv,
                                          const int* num_splits, int max_splits, DecItem& it) {
   const int G = Hq / Hkv, npass = G / GT, NG = Hkv * npass;
   const long long per_c = static_cast<long long>(N) * NG;
   const int c = static_cast<int>(idx / per_c);
   const int r = static_cast<int>(idx - c * per_c);
   const int n = r / NG, gi = r - (r / NG) * NG;
-  const int start = offsets[n];
-  const int L = offsets[n + 1] - start;
+  int start, L;
+  dec_stream(kv, n, start, L);
   const int C_n = stream_splits(num_splits, n, L, max_splits);
   if (c >= C_n) return false;
-  dec_item_fill<GT>(n, c, gi, start, L, C_n, Hq, Hkv, it);
+  dec_item_fill<GT>(n, c, gi, start, L, C_n, Hq, Hkv, kv.block_table != nullptr, it);
   return true;
 }
 
@@ -167,7 +197,7 @@ template <int D, int GT>
 __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
-                        const uint16_t* __restrict__ v, const int* __restrict__ offsets, int N,
+                        const uint16_t* __restrict__ v, const DecKV kv, int N,
                         const int* __restrict__ num_splits, int max_splits, int Hq, int Hkv, float scale_log2,
                         float* __restrict__ part_o, float* __restrict__ part_ml, int* status) {
   using C = DecCfg<D>;
@@ -197,7 +227,11 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
     for (int n0 = 0; n0 < N; n0 += 32) {
       const int n = n0 + lane;
       int cnt = 0;
-      if (n < N) cnt = NG * stream_splits(num_splits, n, offsets[n + 1] - offsets[n], max_splits);
+      if (n < N) {
+        int st0, L;
+        dec_stream(kv, n, st0, L);
+        cnt = NG * stream_splits(num_splits, n, L, max_splits);
+      }
       int incl = cnt;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -226,15 +260,16 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
   // item number i of the walk -> item; false for a sparse slot past its stream's split count
   auto next_item = [&](long long i, DecItem& it) -> bool {
     if (dense) {
-      dec_item_dense<GT>(static_cast<int>(i), N, Hq, Hkv, offsets, base, it);
+      dec_item_dense<GT>(static_cast<int>(i), N, Hq, Hkv, kv, base, it);
       return true;
     }
-    return dec_item<GT>(i, N, Hq, Hkv, offsets, num_splits, max_splits, it);
+    return dec_item<GT>(i, N, Hq, Hkv, kv, num_splits, max_splits, it);
   };
 
   if (warp == 4) {
     // ---------------------------------------------------------------- producer
-    const int T = min(offsets[N], kDecMapRows);  // no box may reach past the cache
+    const bool paged = kv.block_table != nullptr;
+    const int T = paged ? 0 : min(kv.offsets[N], kDecMapRows);  // no box may reach past the cache
     const long long rs = static_cast<long long>(Hkv) * D;
     long long gb = 0;  // ring position: blocks issued so far
     int qi = 0;        // items started so far
@@ -255,9 +290,23 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
       ++qi;
       for (int bk = 0; bk < it.nblk; ++bk) {
         const int s = static_cast<int>(gb % kDecStages);
-        const int row0 = it.start + it.k0 + bk * kDecBlk;
-        const bool tile = row0 + kDecBlk <= T;
-        const int nrows = tile ? kDecBlk : min(kDecBlk, it.k1 - (it.k0 + bk * kDecBlk));
+        const int t0 = it.k0 + bk * kDecBlk;  // the block's first key in the stream
+        int row0, nrows;
+        bool tile;
+        if (paged) {
+          // chunks are whole blocks, so the block lies in one page; a full box is copied only when all
+          // of its rows are keys of the stream (the rest of a last page may hold anything)
+          const int page = kv.block_table[static_cast<long long>(it.n) * kv.max_pages + t0 / kv.page_size];
+          const bool page_ok = page >= 0 && page < kv.num_pages;
+          if (!page_ok && lane == 0) record_status(status, kStatusBadArg);
+          row0 = page_ok ? page * kv.page_size + t0 % kv.page_size : 0;
+          tile = page_ok && t0 + kDecBlk <= it.k1;
+          nrows = page_ok ? min(kDecBlk, it.k1 - t0) : 0;  // an invalid page is read as zeros
+        } else {
+          row0 = it.start + t0;
+          tile = row0 + kDecBlk <= T;
+          nrows = tile ? kDecBlk : min(kDecBlk, it.k1 - t0);
+        }
         if (lane == 0) ok = mbar_wait(empty + s, static_cast<uint32_t>((gb / kDecStages) & 1) ^ 1, abort, status);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
@@ -455,7 +504,7 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
 template <int D>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __restrict__ part_o,
                                                              const float* __restrict__ part_ml,
-                                                             const int* __restrict__ offsets,
+                                                             const DecKV kv,
                                                              const int* __restrict__ num_splits, int max_splits,
                                                              int N, int Hq, uint16_t* __restrict__ o,
                                                              float* __restrict__ lse) {
@@ -465,7 +514,8 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
   const long long gw = static_cast<long long>(blockIdx.x) * 4 + warp;
   if (gw >= static_cast<long long>(N) * Hq) return;
   const int n = static_cast<int>(gw / Hq), h = static_cast<int>(gw % Hq);
-  const int L = offsets[n + 1] - offsets[n];
+  int st0, L;
+  dec_stream(kv, n, st0, L);
   const int C = stream_splits(num_splits, n, L, max_splits);
   const long long slot0 = (static_cast<long long>(n) * Hq + h) * max_splits;
   // The first 16 partial rows are loaded before anything else, so their loads and those of the
@@ -546,7 +596,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
 
 template <int D, int GT>
 cudaError_t launch_split(const DecodeProblem& p, const void* q, const void* k, const void* v,
-                         const CUtensorMap& mk, const CUtensorMap& mv, const int* offsets, const int* num_splits,
+                         const CUtensorMap& mk, const CUtensorMap& mv, const DecKV& kv, const int* num_splits,
                          float* part_o, float* part_ml, cudaStream_t st) {
   using C = DecCfg<D>;
   const int npass = (p.Hq / p.Hkv) / GT;
@@ -565,41 +615,42 @@ cudaError_t launch_split(const DecodeProblem& p, const void* q, const void* k, c
     LaunchScope ls("decode_split", st);
     decode_split_kernel<D, GT><<<grid, kDecThreads, C::kSmemBytes, st>>>(
         mk, mv, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v),
-        offsets, p.N, num_splits, p.max_splits, p.Hq, p.Hkv, p.scale * kLog2e, part_o, part_ml,
+        kv, p.N, num_splits, p.max_splits, p.Hq, p.Hkv, p.scale * kLog2e, part_o, part_ml,
         device_status_ptr());
   }
   return cudaGetLastError();
 }
 
 template <int D>
-cudaError_t launch_decode_d(const DecodeProblem& p, const void* q, const void* k, const void* v,
-                            const int* offsets, const int* num_splits, void* o, float* lse, void* workspace,
+cudaError_t launch_decode_d(const DecodeProblem& p, const void* q, const void* k, const void* v, const DecKV& kv,
+                            long long map_rows, const int* num_splits, void* o, float* lse, void* workspace,
                             cudaStream_t st) {
   const size_t slots = static_cast<size_t>(p.N) * p.Hq * p.max_splits;
   float* part_o = static_cast<float*>(workspace);
   float* part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                             ((slots * D * sizeof(float) + 255) & ~static_cast<size_t>(255)));
-  // K and V as 3-D maps (D, Hkv, rows) over the packed caches. The row extent is nominal (the real
-  // count is on the device); the kernel never issues a box that reaches past kv_offsets[N].
+  // K and V as 3-D maps (D, Hkv, rows) over the packed caches or the page pool. For packed caches
+  // the row extent is nominal (the real count is on the device) and the kernel never issues a box
+  // that reaches past kv_offsets[N]; a pool's extent is its real row count.
   CUtensorMap mk, mv;
-  if (!make_map_packed_bf16(&mk, k, kDecMapRows, p.Hkv, D, kDecBlk) ||
-      !make_map_packed_bf16(&mv, v, kDecMapRows, p.Hkv, D, kDecBlk))
+  if (!make_map_packed_bf16(&mk, k, map_rows, p.Hkv, D, kDecBlk) ||
+      !make_map_packed_bf16(&mv, v, map_rows, p.Hkv, D, kDecBlk))
     return cudaErrorInvalidValue;
   const int G = p.Hq / p.Hkv;
   cudaError_t e;
   if (G % 4 == 0)  // at most four query heads per CTA
-    e = launch_split<D, 4>(p, q, k, v, mk, mv, offsets, num_splits, part_o, part_ml, st);
+    e = launch_split<D, 4>(p, q, k, v, mk, mv, kv, num_splits, part_o, part_ml, st);
   else if (G % 2 == 0)
-    e = launch_split<D, 2>(p, q, k, v, mk, mv, offsets, num_splits, part_o, part_ml, st);
+    e = launch_split<D, 2>(p, q, k, v, mk, mv, kv, num_splits, part_o, part_ml, st);
   else
-    e = launch_split<D, 1>(p, q, k, v, mk, mv, offsets, num_splits, part_o, part_ml, st);
+    e = launch_split<D, 1>(p, q, k, v, mk, mv, kv, num_splits, part_o, part_ml, st);
   if (e != cudaSuccess) return e;
   const long long warps = static_cast<long long>(p.N) * p.Hq;
   {
     LaunchScope ls("decode_combine", st);
     const cudaError_t e2 =
         launch_dependent(decode_combine_kernel<D>, dim3(static_cast<unsigned>((warps + 3) / 4)), dim3(128), 0, st,
-                         part_o, part_ml, offsets, num_splits, p.max_splits, p.N, p.Hq, static_cast<uint16_t*>(o), lse);
+                         part_o, part_ml, kv, num_splits, p.max_splits, p.N, p.Hq, static_cast<uint16_t*>(o), lse);
     if (e2 != cudaSuccess) return e2;
   }
   return cudaGetLastError();
@@ -610,8 +661,19 @@ cudaError_t launch_decode_d(const DecodeProblem& p, const void* q, const void* k
 cudaError_t launch_decode(const DecodeProblem& p, const void* q, const void* k, const void* v,
                           const int* kv_offsets, const int* num_splits, void* o, float* lse, void* workspace,
                           cudaStream_t st) {
-  if (p.D == 128) return launch_decode_d<128>(p, q, k, v, kv_offsets, num_splits, o, lse, workspace, st);
-  return launch_decode_d<64>(p, q, k, v, kv_offsets, num_splits, o, lse, workspace, st);
+  const DecKV kv{kv_offsets, nullptr, nullptr, 0, 0, 0};
+  if (p.D == 128) return launch_decode_d<128>(p, q, k, v, kv, kDecMapRows, num_splits, o, lse, workspace, st);
+  return launch_decode_d<64>(p, q, k, v, kv, kDecMapRows, num_splits, o, lse, workspace, st);
+}
+
+cudaError_t launch_decode_paged(const DecodeProblem& p, const void* q, const void* k_pages, const void* v_pages,
+                                const int* block_table, int max_pages, const int* seq_lens, int page_size,
+                                int num_pages, const int* num_splits, void* o, float* lse, void* workspace,
+                                cudaStream_t st) {
+  const DecKV kv{nullptr, seq_lens, block_table, max_pages, page_size, num_pages};
+  const long long rows = static_cast<long long>(num_pages) * page_size;
+  if (p.D == 128) return launch_decode_d<128>(p, q, k_pages, v_pages, kv, rows, num_splits, o, lse, workspace, st);
+  return launch_decode_d<64>(p, q, k_pages, v_pages, kv, rows, num_splits, o, lse, workspace, st);
 }
 
 }  // namespace attn

@@ -70,6 +70,13 @@ int decode_default_splits(int L, int max_splits);
 cudaError_t launch_decode(const DecodeProblem& p, const void* q, const void* k, const void* v,
                           const int* kv_offsets, const int* num_splits, void* o, float* lse, void* workspace,
                           cudaStream_t st);
+// The same split + combine over a paged cache: key t of stream n is row t % page_size of page
+// block_table[n * max_pages + t / page_size] of the pools k_pages / v_pages [num_pages, page_size,
+// Hkv, D]; stream n has seq_lens[n] keys. page_size is a multiple of 16.
+cudaError_t launch_decode_paged(const DecodeProblem& p, const void* q, const void* k_pages, const void* v_pages,
+                                const int* block_table, int max_pages, const int* seq_lens, int page_size,
+                                int num_pages, const int* num_splits, void* o, float* lse, void* workspace,
+                                cudaStream_t st);
 
 // fwd_sm100.cu: tcgen05 / TMA forward, bf16, D in {64, 128}.
 cudaError_t launch_fwd_sm100(const Problem& p, const void* q, const void* k, const void* v, void* o, float* lse,

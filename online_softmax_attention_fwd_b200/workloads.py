@@ -11,6 +11,8 @@ values. Each workload is named for what it is and its sizes, after the workloads
   D=128), standing in for the Qwen3-8B decode graph of the same paragraph.
 * ``decode48``: 48 decode streams (Hq=32, Hkv=8, D=128), per-stream cache lengths uniform in
   [1024, 4096], packed, the 48-stream decode step of the third paragraph.
+* ``paged_from_packed``: a decode batch's caches laid out in fixed-size pages of a shuffled pool with
+  a block table (a serving engine's paged cache); unused pool rows hold NaN.
 * ``long_prefill_44k``: one 44032-token causal prefill (Hq=32, Hkv=8, D=128) with 1 % of keys given
   a +4.0 shift on one random dimension per key, the 44k-token time-to-first-token case of the third
   paragraph. No dataset or trained weight is used anywhere.
@@ -155,6 +157,49 @@ def random_decode(N, Hq, Hkv, D, lengths, seed=0, dtype=torch.bfloat16, name=Non
     return Decode(name or f"decode_n{N}_hq{Hq}_hkv{Hkv}_d{D}", q.to(dtype), k.to(dtype),
                   v.to(dtype), offsets.to(torch.int32), 1.0 / math.sqrt(D),
                   meta=dict(lengths=lengths))
+
+
+@dataclass
+class PagedCache:
+    k_pages: torch.Tensor      # [num_pages, page_size, Hkv, D]
+    v_pages: torch.Tensor      # [num_pages, page_size, Hkv, D]
+    block_table: torch.Tensor  # [N, max_pages] int32 page ids (-1 where a stream has no page)
+    seq_lens: torch.Tensor     # [N] int32
+
+
+def paged_from_packed(w: Decode, page_size: int, seed: int = 0, spare_pages: int = 3,
+                      fill: float = float("nan")) -> PagedCache:
+    """The same caches as ``w`` laid out in pages of ``page_size`` rows in a shuffled pool.
+
+    Stream n's key t goes to row t % page_size of its (t // page_size)-th page; the pages of all
+    streams, plus ``spare_pages`` unused ones, take a random order in the pool (seeded). Pool rows
+    that hold no key (the rest of a stream's last page, and the spare pages) are set to ``fill``
+    (NaN by default), so that reading one shows up in the result.
+    """
+    g = _gen(seed)
+    off = w.offsets.to(torch.int64)
+    N = off.numel() - 1
+    lens = off[1:] - off[:-1]
+    npg = (lens + page_size - 1) // page_size
+    total = int(npg.sum()) + spare_pages
+    perm = torch.randperm(total, generator=g)
+    Hkv, D = w.k.shape[1], w.k.shape[2]
+    kp = torch.full((total, page_size, Hkv, D), fill, dtype=w.k.dtype)
+    vp = torch.full((total, page_size, Hkv, D), fill, dtype=w.v.dtype)
+    max_pages = max(1, int(npg.max()) if N > 0 else 1)
+    table = torch.full((N, max_pages), -1, dtype=torch.int32)
+    nxt = 0
+    for n in range(N):
+        s0 = int(off[n])
+        for i in range(int(npg[n])):
+            page = int(perm[nxt])
+            nxt += 1
+            table[n, i] = page
+            r0 = i * page_size
+            r1 = min(int(lens[n]), r0 + page_size)
+            kp[page, : r1 - r0] = w.k[s0 + r0: s0 + r1]
+            vp[page, : r1 - r0] = w.v[s0 + r0: s0 + r1]
+    return PagedCache(kp, vp, table, lens.to(torch.int32))
 
 
 def decode48(N: int = 48, lo: int = 1024, hi: int = 4096) -> Decode:

@@ -20,6 +20,8 @@ from .attention import (  # noqa: F401
     attention_fwd_rows,
     attention_bwd,
     decode_attention,
+    decode_attention_paged,
+    paged_rows,
     monoid_identity,
     monoid_leaf,
     monoid_merge,

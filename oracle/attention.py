@@ -22,7 +22,8 @@ No formula is printed on any page. Readings taken (each listed in the design doc):
     identity (-inf, 0, 0), and e^{-inf - M} taken as 0 so no inf - inf is ever formed.
 
 Layouts (row-major): Q, O, dO, dQ are [B, Sq, Hq, D]; K, V, dK, dV are [B, Sk, Hkv, D]; lse is
-[B, Hq, Sq]. Decode: q [N, Hq, D], packed k, v [T, Hkv, D], offsets [N + 1].
+[B, Hq, Sq]. Decode: q [N, Hq, D], packed k, v [T, Hkv, D], offsets [N + 1]; or a paged cache:
+pools [num_pages, page_size, Hkv, D], block_table [N, max_pages], seq_lens [N].
 
 The attention functions use the explicit two-pass softmax (pass 1: the row max; pass 2: the
 exponentials, their sum and the weighted sum of V). The monoid functions exist for the algebra
@@ -226,6 +227,35 @@ def decode_attention(q, k, v, offsets, scale: float):
             o[n, h, :] = (w / Z) @ v[s:e, g, :]
             lse[n, h] = M + math.log(Z)
     return o, lse
+
+
+def paged_rows(block_table, seq_lens, page_size: int):
+    """The pool (page, row) of every key of every stream of a paged cache, by its definition: key t
+    of stream n is row t % page_size of page block_table[n, t // page_size]. Returns one pair of
+    index arrays (pages [L_n], rows [L_n]) per stream; only the table entries of pages that hold
+    keys are read."""
+    bt = np.asarray(block_table, dtype=np.int64)
+    out = []
+    for n, L in enumerate(np.asarray(seq_lens, dtype=np.int64)):
+        t = np.arange(int(L), dtype=np.int64)
+        out.append((bt[n, t // page_size], t % page_size))
+    return out
+
+
+def decode_attention_paged(q, k_pages, v_pages, block_table, seq_lens, scale: float):
+    """Decode attention over a paged cache: the keys and values of each stream are gathered from
+    the pool [num_pages, page_size, Hkv, D] in key order (``paged_rows``), and the result is
+    ``decode_attention`` of that packed cache. Pool rows that hold no key are never read."""
+    k_pages, v_pages = _f64(k_pages), _f64(v_pages)
+    idx = paged_rows(block_table, seq_lens, k_pages.shape[1])
+    ks = [k_pages[p, r] for p, r in idx]
+    vs = [v_pages[p, r] for p, r in idx]
+    Hkv, D = k_pages.shape[2], k_pages.shape[3]
+    k = np.concatenate(ks, axis=0) if ks else np.zeros((0, Hkv, D))
+    v = np.concatenate(vs, axis=0) if vs else np.zeros((0, Hkv, D))
+    off = np.zeros(len(idx) + 1, dtype=np.int64)
+    off[1:] = np.cumsum([len(p) for p, _ in idx])
+    return decode_attention(q, k, v, off, scale)
 
 
 # ---------------------------------------------------------------------------------------------

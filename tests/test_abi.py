@@ -94,6 +94,30 @@ def test_decode_argument_errors(L):
     assert call(ws=None) == 4
 
 
+def test_paged_decode_argument_errors(L):
+    ws = L.attn_decode_workspace_size(4, 8, 128, 16)
+    base = dict(bt=A, max_pages=8, lens=A, page_size=64, num_pages=100, max_splits=16, N=4, Hq=8, Hkv=2,
+                D=128, ws=A, wsb=ws)
+
+    def call(**kw):
+        a = {**base, **kw}
+        return L.attn_decode_paged(A, A, A, a["bt"], a["max_pages"], a["lens"], a["page_size"], a["num_pages"],
+                                   None, a["max_splits"], A, A, a["N"], a["Hq"], a["Hkv"], a["D"], 0.1, a["ws"],
+                                   a["wsb"], None)
+    assert call(page_size=8) == 1          # below one 16-key block
+    assert call(page_size=24) == 1         # not a multiple of 16
+    assert call(num_pages=0) == 1
+    assert call(max_pages=0) == 1
+    assert call(num_pages=1 << 26, page_size=64) == 1   # pool rows past 2^31
+    assert call(lens=None) == 1
+    assert call(bt=None) == 1
+    assert call(bt=U) == 3
+    assert call(lens=U) == 3
+    assert call(Hq=6, Hkv=4) == 1
+    assert call(D=80) == 2
+    assert call(wsb=ws - 1) == 4
+
+
 def test_launch_counter_and_last_path_without_gpu(L):
     assert attn.launch_count() >= 0
     assert isinstance(attn.last_path(0), str)

@@ -77,3 +77,80 @@ def test_empty_stream_gives_zero_and_minus_inf():
     o, lse = run_decode(w)
     assert np.all(o[0] == 0) and np.all(o[2] == 0)
     assert np.all(np.isneginf(lse[0])) and np.all(np.isneginf(lse[2]))
+
+
+# ---------------------------------------------------------------------------------------------
+# Paged caches (attn_decode_paged): the same streams read through a block table from a shuffled
+# pool whose unused rows are NaN.
+# ---------------------------------------------------------------------------------------------
+
+def run_paged(w, page_size, seed=0, num_splits=None, max_splits=16, block_table=None):
+    dev = torch.device("cuda")
+    pc = W.paged_from_packed(w, page_size, seed=seed)
+    bt = pc.block_table if block_table is None else block_table
+    q, kp, vp, bt_d, sl = (t.to(dev) for t in (w.q, pc.k_pages, pc.v_pages, bt, pc.seq_lens))
+    ns = None if num_splits is None else torch.as_tensor(num_splits, dtype=torch.int32, device=dev)
+    o, lse = attn.decode_paged(q, kp, vp, bt_d, sl, num_splits=ns, max_splits=max_splits, scale=w.scale)
+    torch.cuda.synchronize()
+    return np64(o), np64(lse), pc
+
+
+def ref_paged(w, pc):
+    return oracle.decode_attention_paged(np64(w.q), np64(pc.k_pages), np64(pc.v_pages), pc.block_table.numpy(),
+                                         pc.seq_lens.numpy(), w.scale)
+
+
+@pytest.mark.parametrize("lengths,Hq,Hkv,D,page", [
+    ([1, 2, 15, 16, 17, 0, 1000, 257], 8, 2, 128, 16),   # block-sized pages, empty and 1-key streams
+    ([4096, 1, 513, 64, 65], 32, 8, 128, 64),
+    ([300, 7000, 64], 16, 1, 64, 256),                    # G = 16
+    ([100, 200, 31], 6, 3, 64, 32),                       # G = 2
+    ([129, 31, 256], 3, 3, 128, 128),                     # G = 1
+])
+def test_decode_paged_shapes(lengths, Hq, Hkv, D, page):
+    w = W.random_decode(len(lengths), Hq, Hkv, D, lengths, seed=sum(lengths) + page)
+    o, lse, pc = run_paged(w, page, seed=page)
+    assert attn.device_status() == 0
+    assert attn.last_path(2) == "decode_splitkv_paged_mma16816"
+    assert np.all(np.isfinite(o))                         # no NaN pool row was read
+    o_ref, lse_ref = ref_paged(w, pc)
+    assert_o_bf16(o, o_ref)
+    assert_lse(lse, lse_ref)
+
+
+def test_decode48_paged_matches_packed_oracle():
+    w = W.decode48()
+    o, lse, _ = run_paged(w, 64, seed=3)
+    assert attn.device_status() == 0
+    o_ref, lse_ref = ref(w)                               # the same keys, packed
+    assert_o_bf16(o, o_ref)
+    assert_lse(lse, lse_ref)
+
+
+def test_decode_paged_split_counts_change_rounding_only():
+    w = W.random_decode(5, 8, 2, 128, [3000, 1500, 17, 4096, 33], seed=12)
+    outs = []
+    for ns in ([1] * 5, [16] * 5, [3, 7, 1, 13, 2], [64] * 5):
+        o, lse, pc = run_paged(w, 32, seed=1, num_splits=ns, max_splits=64)
+        assert attn.device_status() == 0
+        o_ref, lse_ref = ref_paged(w, pc)
+        assert_o_bf16(o, o_ref)
+        assert_lse(lse, lse_ref)
+        outs.append(o)
+    for o in outs[1:]:
+        assert max_abs(o, outs[0]) <= 2e-2
+
+
+def test_decode_paged_bad_page_id_is_reported_not_read():
+    # one table entry points one page past the pool: that page is never read (its keys count as
+    # zeros), the device status says ATTN_ERR_INVALID_ARG, and the other streams are unaffected
+    w = W.random_decode(3, 8, 2, 128, [100, 40, 70], seed=5)
+    pc = W.paged_from_packed(w, 16, seed=1)
+    bt = pc.block_table.clone()
+    bt[1, 1] = pc.k_pages.shape[0]
+    o, lse, _ = run_paged(w, 16, seed=1, block_table=bt)
+    assert attn.device_status() == 1
+    assert attn.device_status() == 0                      # reading clears it
+    o_ref, lse_ref = ref_paged(w, pc)
+    assert_o_bf16(o[[0, 2]], o_ref[[0, 2]])
+    assert_lse(lse[[0, 2]], lse_ref[[0, 2]])

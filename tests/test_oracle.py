@@ -320,6 +320,62 @@ def test_decode_matches_forward_with_one_query():
         np.testing.assert_allclose(lse[n], lf[0, :, 0], atol=1e-12)
 
 
+def check_paged_rows(paged_rows):
+    # pages of 2 rows; stream 0 owns pages 3 then 0 and has 3 keys, stream 1 owns page 1, 1 key,
+    # stream 2 has none (its table row is never read, so it may hold anything)
+    table = np.array([[3, 0], [1, 99], [-7, 42]])
+    idx = paged_rows(table, [3, 1, 0], 2)
+    np.testing.assert_array_equal(idx[0][0], [3, 3, 0])
+    np.testing.assert_array_equal(idx[0][1], [0, 1, 0])
+    np.testing.assert_array_equal(idx[1][0], [1])
+    np.testing.assert_array_equal(idx[1][1], [0])
+    assert len(idx[2][0]) == 0
+
+
+def test_paged_rows_by_hand():
+    check_paged_rows(oracle.paged_rows)
+
+
+def check_paged_decode(decode_paged):
+    # keys written into a shuffled pool by hand (a scatter, the inverse of the oracle's gather);
+    # every pool row that holds no key is NaN and must not reach the result
+    rng = np.random.default_rng(9)
+    P, Hq, Hkv, D = 4, 6, 2, 5
+    lengths = [7, 4, 0, 1, 9]
+    q = rng.standard_normal((len(lengths), Hq, D))
+    keys = [rng.standard_normal((L, Hkv, D)) for L in lengths]
+    vals = [rng.standard_normal((L, Hkv, D)) for L in lengths]
+    need = [(L + P - 1) // P for L in lengths]
+    order = rng.permutation(sum(need) + 2)          # two spare pages
+    kp = np.full((len(order), P, Hkv, D), np.nan)
+    vp = np.full((len(order), P, Hkv, D), np.nan)
+    table = np.full((len(lengths), max(need)), -1)
+    used = 0
+    for n, L in enumerate(lengths):
+        for t in range(L):
+            if t % P == 0:
+                table[n, t // P] = order[used]
+                used += 1
+            kp[table[n, t // P], t % P] = keys[n][t]
+            vp[table[n, t // P], t % P] = vals[n][t]
+    o, lse = decode_paged(q, kp, vp, table, lengths, 0.4)
+    assert np.all(np.isfinite(o))
+    for n, L in enumerate(lengths):
+        if L == 0:
+            np.testing.assert_array_equal(o[n], 0.0)
+            assert np.all(np.isneginf(lse[n]))
+            continue
+        o1 = _torch_sdpa(q[n][None, None], keys[n][None], vals[n][None], False, 0.4)
+        np.testing.assert_allclose(o[n], o1[0, 0], atol=1e-12)
+        for h in range(Hq):
+            x = 0.4 * keys[n][:, h // (Hq // Hkv), :] @ q[n, h]
+            assert abs(lse[n, h] - logsumexp(x)) < 1e-12
+
+
+def test_paged_decode_matches_sdpa_per_stream():
+    check_paged_decode(oracle.decode_attention_paged)
+
+
 # ---------------------------------------------------------------------------------------------
 # Monoid algebra.
 # ---------------------------------------------------------------------------------------------

@@ -132,3 +132,43 @@ def test_monoid_merge_without_rescale_is_caught():
     o, _ = oracle.monoid_finalize(t)
     o_ref, _ = FWD(q[None, None, None], k[None, :, None], v[None, :, None], False, s)
     assert not np.allclose(o, o_ref[0, 0, 0], atol=1e-6)
+
+
+# ---------------------------------------------------------------------------------------------
+# Paged decode: the gather of a stream's keys from its pages.
+# ---------------------------------------------------------------------------------------------
+
+def paged_rows_swapped(block_table, seq_lens, page_size):
+    # page and row index exchanged: page from t % page_size, row from t // page_size
+    bt = np.asarray(block_table, dtype=np.int64)
+    out = []
+    for n, L in enumerate(np.asarray(seq_lens, dtype=np.int64)):
+        t = np.arange(int(L), dtype=np.int64)
+        out.append((bt[n, np.minimum(t % page_size, bt.shape[1] - 1)], t // page_size))
+    return out
+
+
+def paged_rows_first_page_only(block_table, seq_lens, page_size):
+    # every key read from the stream's first page
+    bt = np.asarray(block_table, dtype=np.int64)
+    return [(np.full(int(L), bt[n, 0]), np.arange(int(L)) % page_size)
+            for n, L in enumerate(np.asarray(seq_lens, dtype=np.int64))]
+
+
+def paged_decode_with(rows_fn):
+    def decode(q, k_pages, v_pages, block_table, seq_lens, scale):
+        k_pages, v_pages = np.asarray(k_pages, np.float64), np.asarray(v_pages, np.float64)
+        idx = rows_fn(block_table, seq_lens, k_pages.shape[1])
+        k = np.concatenate([k_pages[p, r] for p, r in idx], axis=0)
+        v = np.concatenate([v_pages[p, r] for p, r in idx], axis=0)
+        off = np.concatenate([[0], np.cumsum([len(p) for p, _ in idx])])
+        return oracle.decode_attention(q, k, v, off, scale)
+    return decode
+
+
+@pytest.mark.parametrize("rows_fn", [paged_rows_swapped, paged_rows_first_page_only])
+def test_paged_pins_catch_gather_mistakes(rows_fn):
+    with pytest.raises(AssertionError):
+        T.check_paged_rows(rows_fn)
+    with pytest.raises(AssertionError):
+        T.check_paged_decode(paged_decode_with(rows_fn))

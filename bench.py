@@ -173,6 +173,39 @@ class ClockSampler:
 # distributed helpers (also exercised by tests/test_multirank.py with gloo on CPU)
 # ------------------------------------------------------------------------------------------------
 
+def roofline_entry(prof: dict, work: dict, peaks: dict, peak_src: str, traffic_fn=None):
+    """The `roofline` object for the kernel with the most live device time.
+
+    prof: kernel family -> (total ms, launches) from the CUDA events; work: family -> (bound,
+    algorithmic FLOPs or bytes per launch, or None when the kernel's work is not counted).
+    achieved = work per launch / mean launch time, frac = achieved / the measured peak. A dominant
+    kernel without a work figure (a CUDA-core kernel, or the decode combine, which comes out on top
+    only under a profiler's serialised timing) gets no achieved figure and no fraction.
+    """
+    if not prof:
+        return None
+    traffic_fn = traffic_fn or ncu_traffic
+    dom = max(prof.items(), key=lambda kv: kv[1][0])[0]
+    ms, nl = prof[dom]
+    per_launch_s = ms / 1e3 / nl
+    bound, wk = work.get(dom, ("unknown", None))
+    traffic = traffic_fn(dom, "gqa4k" if dom.startswith(("fwd", "bwd")) else "decode48")
+    if bound == "tensor" and wk is not None:
+        ach = wk / per_launch_s / 1e12
+        return {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+                "frac_of_sustained": ach / peaks["bf16_tflops_sustained"], "traffic": traffic,
+                "peak_source": f"{peak_src} (burst bf16)", "launch_ms": per_launch_s * 1e3}
+    if bound == "hbm" and wk is not None:
+        ach = wk / per_launch_s / 1e9
+        return {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peak_src,
+                "launch_ms": per_launch_s * 1e3}
+    return {"kernel": dom, "bound": "alu" if bound in ("alu", "unknown") else bound, "achieved": None,
+            "peak": None, "unit": None, "frac": None, "traffic": traffic, "launch_ms": per_launch_s * 1e3,
+            "note": "no algorithmic work figure for this kernel; no roofline fraction is claimed"}
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -417,31 +450,7 @@ def run_ours(args):
     work = {"fwd_sm100": ("tensor", f_fwd), "bwd_sm100": ("tensor", f_bwd),
             "bwd_simt_dq": ("alu", None), "bwd_simt_dkdv": ("alu", None),
             "decode_split": ("hbm", b_dec), "decode_combine": ("hbm", None)}
-    dom = max(prof.items(), key=lambda kv: kv[1][0])[0] if prof else None
-    roofline = None
-    if dom:
-        ms, nl = prof[dom]
-        per_launch_s = ms / 1e3 / nl
-        bound, wk = work.get(dom, ("unknown", None))
-        traffic = ncu_traffic(dom, "gqa4k" if dom.startswith(("fwd", "bwd")) else "decode48")
-        if bound == "tensor" and wk is not None:
-            ach = wk / per_launch_s / 1e12
-            roofline = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
-                        "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
-                        "frac_of_sustained": ach / peaks["bf16_tflops_sustained"], "traffic": traffic,
-                        "peak_source": f"{peak_src} (burst bf16)", "launch_ms": per_launch_s * 1e3}
-        elif bound == "hbm" and wk is not None:
-            ach = wk / per_launch_s / 1e9
-            roofline = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                        "frac": ach / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peak_src,
-                        "launch_ms": per_launch_s * 1e3}
-        else:
-            # a CUDA-core kernel, or one whose work is not counted (the decode combine, which can come
-            # out on top only under a profiler's serialised timing)
-            roofline = {"kernel": dom, "bound": "alu" if bound in ("alu", "unknown") else bound, "achieved": None,
-                        "peak": None, "unit": None, "frac": None, "traffic": traffic,
-                        "launch_ms": per_launch_s * 1e3,
-                        "note": "no algorithmic work figure for this kernel; no roofline fraction is claimed"}
+    roofline = roofline_entry(prof, work, peaks, peak_src)
     kernels = {n: {"total_ms": ms, "launches": nl, "share": ms / max(1e-12, sum(x[0] for x in prof.values()))}
                for n, (ms, nl) in prof.items()}
 

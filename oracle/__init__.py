@@ -21,6 +21,8 @@ from .attention import (  # noqa: F401
     attention_bwd,
     decode_attention,
     decode_attention_paged,
+    decode_attention_qlen,
+    decode_attention_paged_qlen,
     paged_rows,
     monoid_identity,
     monoid_leaf,

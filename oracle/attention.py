@@ -10,7 +10,7 @@ Sources. The pages state the method only in words:
     pass also comes out of rewrites of the same graph.
   * "Tang Project Derives GPU Kernels via IR ..." (aibriefing.imbch.dev), section "Details", fourth
     bullet: the workload includes causal forward passes.
-No formula is printed on any page. Readings taken (each listed in the design doc):
+No formula is printed on any page. Readings taken where the pages are silent:
   * attention is softmax(scale * Q K^T + mask) V, per query head h over key/value head
     g = h // (Hq / Hkv) (grouped-query heads, contiguous groups);
   * the causal mask is bottom-right aligned: query i sees key j iff j <= i + (Sk - Sq);
@@ -256,6 +256,46 @@ def decode_attention_paged(q, k_pages, v_pages, block_table, seq_lens, scale: fl
     off = np.zeros(len(idx) + 1, dtype=np.int64)
     off[1:] = np.cumsum([len(p) for p, _ in idx])
     return decode_attention(q, k, v, off, scale)
+
+
+def decode_attention_qlen(q, k, v, offsets, scale: float):
+    """Decode with several query tokens per stream (a speculative or chunked step): stream n brings
+    q_len new query tokens whose keys are already the newest q_len rows of its L_n cached keys, so
+    token t sits at position L_n - q_len + t and sees keys 0 .. L_n - q_len + t. That is the causal
+    forward with Sq = q_len and Sk = L_n under the bottom-right alignment (``visible_mask``), done
+    stream by stream with ``attention_fwd``. Tokens that see no key (L_n < q_len) get O = 0 and
+    lse = -inf. The decode steps are the 16-48-stream steps of "Não escreva kernels, derive-os"
+    ("Aprofundamento", third paragraph); a step with more than one token per stream is this
+    library's reading of the same step for speculative decoding.
+    q [N, q_len, Hq, D]; packed k, v [T, Hkv, D]; offsets [N + 1].
+    Returns (O [N, q_len, Hq, D], lse [N, Hq, q_len])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    off = np.asarray(offsets, dtype=np.int64)
+    N, ql, Hq, D = q.shape
+    o = np.zeros((N, ql, Hq, D), dtype=np.float64)
+    lse = np.full((N, Hq, ql), NEG_INF, dtype=np.float64)
+    for n in range(N):
+        s, e = int(off[n]), int(off[n + 1])
+        if e <= s:
+            continue
+        on, ln = attention_fwd(q[n][None], k[s:e][None], v[s:e][None], True, scale)
+        o[n], lse[n] = on[0], ln[0]
+    return o, lse
+
+
+def decode_attention_paged_qlen(q, k_pages, v_pages, block_table, seq_lens, scale: float):
+    """``decode_attention_qlen`` over a paged cache: each stream's keys and values are gathered from
+    the pool in key order (``paged_rows``) first."""
+    k_pages, v_pages = _f64(k_pages), _f64(v_pages)
+    idx = paged_rows(block_table, seq_lens, k_pages.shape[1])
+    Hkv, D = k_pages.shape[2], k_pages.shape[3]
+    ks = [k_pages[p, r] for p, r in idx]
+    vs = [v_pages[p, r] for p, r in idx]
+    k = np.concatenate(ks, axis=0) if ks else np.zeros((0, Hkv, D))
+    v = np.concatenate(vs, axis=0) if vs else np.zeros((0, Hkv, D))
+    off = np.zeros(len(idx) + 1, dtype=np.int64)
+    off[1:] = np.cumsum([len(p) for p, _ in idx])
+    return decode_attention_qlen(q, k, v, off, scale)
 
 
 # ---------------------------------------------------------------------------------------------

@@ -376,6 +376,98 @@ def test_paged_decode_matches_sdpa_per_stream():
     check_paged_decode(oracle.decode_attention_paged)
 
 
+def check_decode_qlen(decode_qlen):
+    # Several query tokens per stream: token t of a stream with L keys sees keys 0 .. L - q_len + t.
+    # Written here from that definition with scipy's softmax / logsumexp per (stream, token, head),
+    # plus torch's SDPA with the same mask as a boolean tensor.
+    rng = np.random.default_rng(21)
+    ql, Hq, Hkv, D = 3, 4, 2, 5
+    lengths = [6, 3, 2, 0, 9, 1]              # L < q_len: the first tokens see no key
+    off = np.concatenate([[0], np.cumsum(lengths)])
+    q = rng.standard_normal((len(lengths), ql, Hq, D))
+    k = rng.standard_normal((off[-1], Hkv, D))
+    v = rng.standard_normal((off[-1], Hkv, D))
+    o, lse = decode_qlen(q, k, v, off, 0.6)
+    assert o.shape == (len(lengths), ql, Hq, D) and lse.shape == (len(lengths), Hq, ql)
+    for n, L in enumerate(lengths):
+        s = off[n]
+        for t in range(ql):
+            vis = L - ql + t + 1                  # number of keys token t sees
+            for h in range(Hq):
+                g = h // (Hq // Hkv)
+                if vis <= 0:
+                    np.testing.assert_array_equal(o[n, t, h], 0.0)
+                    assert np.isneginf(lse[n, h, t])
+                    continue
+                x = 0.6 * k[s:s + vis, g] @ q[n, t, h]
+                np.testing.assert_allclose(o[n, t, h], softmax(x) @ v[s:s + vis, g], atol=1e-12)
+                assert abs(lse[n, h, t] - logsumexp(x)) < 1e-12
+        if L >= ql:
+            mask = torch.as_tensor(np.arange(L)[None, :] <= (np.arange(ql)[:, None] + L - ql))
+            qt = torch.as_tensor(q[n]).permute(1, 0, 2)[None]                      # [1, Hq, ql, D]
+            kt = torch.as_tensor(k[s:s + L]).repeat_interleave(Hq // Hkv, 1).permute(1, 0, 2)[None]
+            vt = torch.as_tensor(v[s:s + L]).repeat_interleave(Hq // Hkv, 1).permute(1, 0, 2)[None]
+            ref = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=0.6)[0].permute(1, 0, 2)
+            np.testing.assert_allclose(o[n], ref.numpy(), atol=1e-12)
+
+
+def test_decode_qlen_by_definition():
+    check_decode_qlen(oracle.decode_attention_qlen)
+
+
+def test_decode_qlen_one_token_is_decode():
+    rng = np.random.default_rng(22)
+    lengths = [4, 0, 7]
+    off = np.concatenate([[0], np.cumsum(lengths)])
+    q = rng.standard_normal((3, 4, 6))
+    k = rng.standard_normal((off[-1], 2, 6))
+    v = rng.standard_normal((off[-1], 2, 6))
+    o1, l1 = oracle.decode_attention(q, k, v, off, 0.3)
+    o2, l2 = oracle.decode_attention_qlen(q[:, None], k, v, off, 0.3)
+    np.testing.assert_allclose(o2[:, 0], o1, atol=1e-14)
+    np.testing.assert_array_equal(np.isneginf(l2[..., 0]), np.isneginf(l1))
+    np.testing.assert_allclose(np.where(np.isneginf(l1), 0, l2[..., 0]), np.where(np.isneginf(l1), 0, l1), atol=1e-14)
+
+
+def check_paged_decode_qlen(decode_paged_qlen):
+    # the same pool-by-scatter as check_paged_decode, with two query tokens per stream
+    rng = np.random.default_rng(23)
+    P, Hq, Hkv, D, ql = 4, 4, 2, 5, 2
+    lengths = [7, 1, 0, 9]
+    q = rng.standard_normal((len(lengths), ql, Hq, D))
+    keys = [rng.standard_normal((L, Hkv, D)) for L in lengths]
+    vals = [rng.standard_normal((L, Hkv, D)) for L in lengths]
+    need = [(L + P - 1) // P for L in lengths]
+    order = rng.permutation(sum(need) + 1)
+    kp = np.full((len(order), P, Hkv, D), np.nan)
+    vp = np.full((len(order), P, Hkv, D), np.nan)
+    table = np.full((len(lengths), max(need)), -1)
+    used = 0
+    for n, L in enumerate(lengths):
+        for t in range(L):
+            if t % P == 0:
+                table[n, t // P] = order[used]
+                used += 1
+            kp[table[n, t // P], t % P] = keys[n][t]
+            vp[table[n, t // P], t % P] = vals[n][t]
+    o, lse = decode_paged_qlen(q, kp, vp, table, lengths, 0.4)
+    assert np.all(np.isfinite(o))
+    for n, L in enumerate(lengths):
+        for t in range(ql):
+            vis = L - ql + t + 1
+            for h in range(Hq):
+                if vis <= 0:
+                    assert np.all(o[n, t, h] == 0) and np.isneginf(lse[n, h, t])
+                    continue
+                x = 0.4 * keys[n][:vis, h // (Hq // Hkv)] @ q[n, t, h]
+                np.testing.assert_allclose(o[n, t, h], softmax(x) @ vals[n][:vis, h // (Hq // Hkv)], atol=1e-12)
+                assert abs(lse[n, h, t] - logsumexp(x)) < 1e-12
+
+
+def test_paged_decode_qlen_by_definition():
+    check_paged_decode_qlen(oracle.decode_attention_paged_qlen)
+
+
 # ---------------------------------------------------------------------------------------------
 # Monoid algebra.
 # ---------------------------------------------------------------------------------------------

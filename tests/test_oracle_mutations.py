@@ -172,3 +172,39 @@ def test_paged_pins_catch_gather_mistakes(rows_fn):
         T.check_paged_rows(rows_fn)
     with pytest.raises(AssertionError):
         T.check_paged_decode(paged_decode_with(rows_fn))
+
+
+def decode_qlen_top_left(q, k, v, offsets, scale):
+    # Several tokens per stream with the mask aligned to the top-left corner (token t sees keys
+    # 0 .. t) instead of the newest positions.
+    off = np.asarray(offsets)
+    N, ql, Hq, D = q.shape
+    o = np.zeros((N, ql, Hq, D))
+    lse = np.full((N, Hq, ql), -np.inf)
+    for n in range(N):
+        s, e = off[n], off[n + 1]
+        if e <= s:
+            continue
+        L = e - s
+        qq = np.concatenate([q[n], np.zeros((max(0, L - ql), Hq, D))], axis=0)[None] if L > ql else q[n][None]
+        on, ln = oracle.attention_fwd(qq, k[None, s:e], v[None, s:e], True, scale)
+        o[n], lse[n] = on[0, :ql], ln[0, :, :ql]
+    return o, lse
+
+
+def decode_qlen_last_token_for_all(q, k, v, offsets, scale):
+    # every token sees the whole cache (the causal mask among the new tokens forgotten)
+    off = np.asarray(offsets)
+    N, ql, Hq, D = q.shape
+    o = np.zeros((N, ql, Hq, D))
+    lse = np.full((N, Hq, ql), -np.inf)
+    for t in range(ql):
+        ot, lt = oracle.decode_attention(q[:, t], k, v, off, scale)
+        o[:, t], lse[:, :, t] = ot, lt
+    return o, lse
+
+
+@pytest.mark.parametrize("bad", [decode_qlen_top_left, decode_qlen_last_token_for_all])
+def test_decode_qlen_mistakes_are_caught(bad):
+    with pytest.raises(AssertionError):
+        T.check_decode_qlen(bad)

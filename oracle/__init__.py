@@ -19,6 +19,8 @@ from .attention import (  # noqa: F401
     attention_fwd,
     attention_fwd_rows,
     attention_bwd,
+    attention_fwd_varlen,
+    attention_bwd_varlen,
     decode_attention,
     decode_attention_paged,
     decode_attention_qlen,

@@ -198,6 +198,45 @@ def attention_bwd(q, k, v, do, causal: bool, scale: float):
     return dq, dk, dv
 
 
+def attention_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, causal: bool, scale: float):
+    """Forward attention over a packed batch of sequences of different lengths (the multi-stream
+    prefill behind the 44k-token time to first token of "Não escreva kernels, derive-os",
+    "Aprofundamento", third paragraph): sequence b owns query rows cu_q[b] .. cu_q[b+1] - 1 and
+    key/value rows cu_k[b] .. cu_k[b+1] - 1, and attends only to its own keys (causal: bottom-right
+    aligned within the sequence). Each sequence is ``attention_fwd`` with B = 1 on its slices.
+    q [Tq, Hq, D]; k, v [Tk, Hkv, D]. Returns (O [Tq, Hq, D], lse [Hq, Tq])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cq = np.asarray(cu_seqlens_q, dtype=np.int64)
+    ck = np.asarray(cu_seqlens_k, dtype=np.int64)
+    Tq, Hq, D = q.shape
+    o = np.zeros((Tq, Hq, v.shape[2]), dtype=np.float64)
+    lse = np.full((Hq, Tq), NEG_INF, dtype=np.float64)
+    for b in range(len(cq) - 1):
+        q0, q1, k0, k1 = int(cq[b]), int(cq[b + 1]), int(ck[b]), int(ck[b + 1])
+        if q1 <= q0 or k1 <= k0:
+            continue                      # no query rows, or no key: O = 0, lse = -inf
+        ob, lb = attention_fwd(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], causal, scale)
+        o[q0:q1] = ob[0]
+        lse[:, q0:q1] = lb[0]
+    return o, lse
+
+
+def attention_bwd_varlen(q, k, v, do, cu_seqlens_q, cu_seqlens_k, causal: bool, scale: float):
+    """Backward of ``attention_fwd_varlen``: ``attention_bwd`` on each sequence's slices; keys of
+    a sequence that no query row sees get dK = dV = 0. Returns (dQ [Tq,Hq,D], dK, dV [Tk,Hkv,D])."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    cq = np.asarray(cu_seqlens_q, dtype=np.int64)
+    ck = np.asarray(cu_seqlens_k, dtype=np.int64)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for b in range(len(cq) - 1):
+        q0, q1, k0, k1 = int(cq[b]), int(cq[b + 1]), int(ck[b]), int(ck[b + 1])
+        if q1 <= q0 or k1 <= k0:
+            continue
+        gq, gk, gv = attention_bwd(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], do[None, q0:q1], causal, scale)
+        dq[q0:q1], dk[k0:k1], dv[k0:k1] = gq[0], gk[0], gv[0]
+    return dq, dk, dv
+
+
 def decode_attention(q, k, v, offsets, scale: float):
     """Decode attention: stream n's single query attends all L_n = off[n+1] - off[n] of its keys.
 

@@ -468,6 +468,84 @@ def test_paged_decode_qlen_by_definition():
     check_paged_decode_qlen(oracle.decode_attention_paged_qlen)
 
 
+def check_varlen(fwd_varlen, bwd_varlen):
+    # Packed sequences of different lengths. Pins: (1) a batch of equal lengths equals the padded
+    # batch's torch SDPA (bottom-right causal, GQA by repeating kv heads); (2) every sequence equals
+    # torch SDPA on its own slices, so no sequence sees another's keys; (3) a sequence with no key
+    # or no query row contributes nothing and its rows get O = 0, lse = -inf; (4) the gradients
+    # match central finite differences of the packed forward on a tiny case.
+    rng = np.random.default_rng(31)
+    Hq, Hkv, D = 4, 2, 3
+    lq = [3, 0, 5, 2, 4]
+    lk = [5, 2, 5, 0, 4]
+    cq = np.concatenate([[0], np.cumsum(lq)])
+    ck = np.concatenate([[0], np.cumsum(lk)])
+    q = rng.standard_normal((cq[-1], Hq, D))
+    k = rng.standard_normal((ck[-1], Hkv, D))
+    v = rng.standard_normal((ck[-1], Hkv, D))
+    do = rng.standard_normal((cq[-1], Hq, D))
+    for causal in (False, True):
+        o, lse = fwd_varlen(q, k, v, cq, ck, causal, 0.7)
+        assert o.shape == q.shape and lse.shape == (Hq, cq[-1])
+        for b in range(len(lq)):
+            rows = slice(cq[b], cq[b + 1])
+            if lq[b] == 0:
+                continue
+            if lk[b] == 0:
+                assert np.all(o[rows] == 0) and np.all(np.isneginf(lse[:, rows]))
+                continue
+            # torch's is_causal is top-left aligned; the bottom-right mask goes in as a boolean tensor
+            mask = torch.as_tensor(np.arange(lk[b])[None] <= np.arange(lq[b])[:, None] + lk[b] - lq[b]) \
+                if causal else None
+            t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).permute(1, 0, 2)[None]
+            ref = F.scaled_dot_product_attention(t(q[rows]), t(k[ck[b]:ck[b + 1]]), t(v[ck[b]:ck[b + 1]]),
+                                                 attn_mask=mask, scale=0.7, enable_gqa=True)
+            np.testing.assert_allclose(o[rows], ref[0].permute(1, 0, 2).numpy(), atol=1e-12)
+            for h in range(Hq):
+                x = 0.7 * q[rows, h] @ k[ck[b]:ck[b + 1], h // 2].T
+                if causal:
+                    x = np.where(np.arange(lk[b])[None] <= np.arange(lq[b])[:, None] + lk[b] - lq[b], x, -np.inf)
+                with np.errstate(divide="ignore"):
+                    want = logsumexp(x, axis=1)
+                np.testing.assert_allclose(lse[h, rows], want, atol=1e-12)
+    # finite differences of sum(O * dO) on the packed batch
+    causal = True
+    dq, dk, dv = bwd_varlen(q, k, v, do, cq, ck, causal, 0.7)
+    f = lambda qq, kk, vv: float(np.sum(fwd_varlen(qq, kk, vv, cq, ck, causal, 0.7)[0] * do))
+    eps = 1e-6
+    for arr, grad in ((q, dq), (k, dk), (v, dv)):
+        for idx in [(0, 0, 0), (arr.shape[0] - 1, 1, 2), (arr.shape[0] // 2, arr.shape[1] - 1, 1)]:
+            a1, a2 = arr.copy(), arr.copy()
+            a1[idx] += eps
+            a2[idx] -= eps
+            args1 = [a1 if arr is x else x for x in (q, k, v)]
+            args2 = [a2 if arr is x else x for x in (q, k, v)]
+            fd = (f(*args1) - f(*args2)) / (2 * eps)
+            assert abs(fd - grad[idx]) < 1e-6 * max(1.0, abs(fd)), (idx, fd, grad[idx])
+
+
+def test_varlen_by_definition():
+    check_varlen(oracle.attention_fwd_varlen, oracle.attention_bwd_varlen)
+
+
+def test_varlen_equal_lengths_is_the_dense_batch():
+    rng = np.random.default_rng(32)
+    B, S, Hq, Hkv, D = 3, 6, 4, 2, 4
+    q, k, v, do = (rng.standard_normal((B, S, H, D)) for H in (Hq, Hkv, Hkv, Hq))
+    cu = np.arange(B + 1) * S
+    for causal in (False, True):
+        o, lse = oracle.attention_fwd_varlen(q.reshape(-1, Hq, D), k.reshape(-1, Hkv, D), v.reshape(-1, Hkv, D),
+                                             cu, cu, causal, 0.5)
+        od, ld = oracle.attention_fwd(q, k, v, causal, 0.5)
+        np.testing.assert_allclose(o, od.reshape(-1, Hq, D), atol=1e-14)
+        np.testing.assert_allclose(lse, ld.transpose(1, 0, 2).reshape(Hq, -1), atol=1e-14)
+        g = oracle.attention_bwd_varlen(q.reshape(-1, Hq, D), k.reshape(-1, Hkv, D), v.reshape(-1, Hkv, D),
+                                        do.reshape(-1, Hq, D), cu, cu, causal, 0.5)
+        gd = oracle.attention_bwd(q, k, v, do, causal, 0.5)
+        for a, b in zip(g, gd):
+            np.testing.assert_allclose(a, b.reshape(a.shape), atol=1e-14)
+
+
 # ---------------------------------------------------------------------------------------------
 # Monoid algebra.
 # ---------------------------------------------------------------------------------------------

@@ -208,3 +208,29 @@ def decode_qlen_last_token_for_all(q, k, v, offsets, scale):
 def test_decode_qlen_mistakes_are_caught(bad):
     with pytest.raises(AssertionError):
         T.check_decode_qlen(bad)
+
+
+def varlen_one_sequence(q, k, v, cq, ck, causal, scale):
+    # the packed rows treated as one long sequence: sequences see each other's keys
+    o, lse = oracle.attention_fwd(q[None], k[None], v[None], causal, scale)
+    return o[0], lse[0]
+
+
+def varlen_bwd_one_sequence(q, k, v, do, cq, ck, causal, scale):
+    g = oracle.attention_bwd(q[None], k[None], v[None], do[None], causal, scale)
+    return tuple(x[0] for x in g)
+
+
+def varlen_bwd_without_dv(q, k, v, do, cq, ck, causal, scale):
+    dq, dk, dv = oracle.attention_bwd_varlen(q, k, v, do, cq, ck, causal, scale)
+    return dq, dk, np.zeros_like(dv)
+
+
+@pytest.mark.parametrize("fwd,bwd", [
+    (varlen_one_sequence, oracle.attention_bwd_varlen),
+    (oracle.attention_fwd_varlen, varlen_bwd_one_sequence),
+    (oracle.attention_fwd_varlen, varlen_bwd_without_dv),
+])
+def test_varlen_mistakes_are_caught(fwd, bwd):
+    with pytest.raises(AssertionError):
+        T.check_varlen(fwd, bwd)

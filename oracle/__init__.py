@@ -20,6 +20,8 @@ from .attention import (  # noqa: F401
     attention_fwd_rows,
     attention_bwd,
     attention_fwd_varlen,
+    attention_fwd_fp8,
+    e4m3_to_float,
     attention_bwd_varlen,
     decode_attention,
     decode_attention_paged,

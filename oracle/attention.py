@@ -237,6 +237,30 @@ def attention_bwd_varlen(q, k, v, do, cu_seqlens_q, cu_seqlens_k, causal: bool, 
     return dq, dk, dv
 
 
+def e4m3_to_float(codes) -> np.ndarray:
+    """Values of 8-bit E4M3 codes (the OCP 8-bit floating-point format with 4 exponent bits, bias 7,
+    and 3 mantissa bits; no infinities, S.1111.111 is NaN): exponent field 0 is subnormal,
+    (-1)^s 2^-6 m/8; otherwise (-1)^s 2^(e-7) (1 + m/8). Largest finite value 448."""
+    c = np.asarray(codes, dtype=np.int64) & 0xFF
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    val = np.where(e == 0, np.ldexp(m / 8.0, -6), np.ldexp(1.0 + m / 8.0, e - 7))
+    val = np.where((e == 15) & (m == 7), np.nan, val)
+    return sign * val
+
+
+def attention_fwd_fp8(q8, k8, v8, q_scale: float, k_scale: float, v_scale: float, causal: bool, scale: float):
+    """Forward attention on 8-bit E4M3 inputs with per-tensor scales (the FP8 checkpoint the third
+    paragraph of "Aprofundamento" credits with a much shorter time to first token): the real inputs
+    are Q = q_scale q8, K = k_scale k8, V = v_scale v8, and the result is ``attention_fwd`` of them.
+    q8 [B, Sq, Hq, D], k8 / v8 [B, Sk, Hkv, D] hold the codes (uint8). Returns (O, lse) in fp64."""
+    q = q_scale * e4m3_to_float(q8)
+    k = k_scale * e4m3_to_float(k8)
+    v = v_scale * e4m3_to_float(v8)
+    return attention_fwd(q, k, v, causal, scale)
+
+
 def decode_attention(q, k, v, offsets, scale: float):
     """Decode attention: stream n's single query attends all L_n = off[n+1] - off[n] of its keys.
 

@@ -546,6 +546,46 @@ def test_varlen_equal_lengths_is_the_dense_batch():
             np.testing.assert_allclose(a, b.reshape(a.shape), atol=1e-14)
 
 
+def check_e4m3(decode):
+    # hand-worked codes, then every code against torch's float8_e4m3fn conversion (a library routine)
+    assert decode(0x38) == 1.0                      # e = 7, m = 0
+    assert decode(0x7E) == 448.0                    # largest finite: 2^8 * 1.75
+    assert decode(0x01) == 2.0 ** -9                # smallest subnormal: 2^-6 * 1/8
+    assert decode(0x08) == 2.0 ** -6                # smallest normal
+    assert decode(0xB8) == -1.0 and decode(0x3C) == 1.5 and decode(0x44) == 3.0
+    assert np.isnan(decode(0x7F)) and np.isnan(decode(0xFF))
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = decode(codes)
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(ref))
+    np.testing.assert_array_equal(got[~np.isnan(ref)], ref[~np.isnan(ref)])
+
+
+def test_e4m3_decoder():
+    check_e4m3(oracle.e4m3_to_float)
+
+
+def check_fp8_attention(fwd8):
+    # the per-tensor scales enter as the real inputs: q_scale and k_scale only through their
+    # product in the scores, v_scale as a factor of O (lse does not depend on it)
+    rng = np.random.default_rng(33)
+    vals = torch.from_numpy(rng.standard_normal((3, 1, 20, 2, 8)))
+    q8, k8, v8 = (x.to(torch.float8_e4m3fn).view(torch.uint8).numpy() for x in vals)
+    dq, dk, dv = (torch.from_numpy(x).view(torch.float8_e4m3fn).to(torch.float64).numpy() for x in (q8, k8, v8))
+    for causal in (False, True):
+        o, lse = fwd8(q8, k8, v8, 0.5, 3.0, 2.0, causal, 0.3)
+        o_ref, lse_ref = oracle.attention_fwd(0.5 * dq, 3.0 * dk, 2.0 * dv, causal, 0.3)
+        np.testing.assert_allclose(o, o_ref, atol=1e-12)
+        np.testing.assert_allclose(lse, lse_ref, atol=1e-12)
+        o2, lse2 = fwd8(q8, k8, v8, 1.5, 1.0, 1.0, causal, 0.3)   # same score scale product
+        np.testing.assert_allclose(o2 * 2.0, o, atol=1e-12)
+        np.testing.assert_allclose(lse2, lse, atol=1e-12)
+
+
+def test_fp8_attention_scales():
+    check_fp8_attention(oracle.attention_fwd_fp8)
+
+
 # ---------------------------------------------------------------------------------------------
 # Monoid algebra.
 # ---------------------------------------------------------------------------------------------

@@ -234,3 +234,28 @@ def varlen_bwd_without_dv(q, k, v, do, cq, ck, causal, scale):
 def test_varlen_mistakes_are_caught(fwd, bwd):
     with pytest.raises(AssertionError):
         T.check_varlen(fwd, bwd)
+
+
+def e4m3_bias_8(codes):
+    return oracle.e4m3_to_float(codes) / 2.0
+
+
+def e4m3_no_subnormals(codes):
+    c = np.asarray(codes, dtype=np.int64) & 0xFF
+    v = oracle.e4m3_to_float(codes)
+    return np.where(((c >> 3) & 0xF) == 0, 0.0 * v, v)
+
+
+@pytest.mark.parametrize("bad", [e4m3_bias_8, e4m3_no_subnormals])
+def test_e4m3_decoder_mistakes_are_caught(bad):
+    with pytest.raises(AssertionError):
+        T.check_e4m3(bad)
+
+
+def fp8_v_scale_on_scores(q8, k8, v8, qs, ks, vs, causal, scale):
+    return oracle.attention_fwd_fp8(q8, k8, v8, qs * vs, ks, 1.0, causal, scale)
+
+
+def test_fp8_scale_mistake_is_caught():
+    with pytest.raises(AssertionError):
+        T.check_fp8_attention(fp8_v_scale_on_scores)

@@ -6,7 +6,7 @@ import torch
 import online_softmax_attention_fwd_b200 as attn
 import oracle
 from online_softmax_attention_fwd_b200 import workloads as W
-from tests._util import assert_lse, assert_o_bf16, np64, max_abs
+from tests._util import assert_lse, assert_o_bf16, np64, max_abs, running_max_moves
 
 pytestmark = pytest.mark.gpu
 
@@ -77,6 +77,92 @@ def test_empty_stream_gives_zero_and_minus_inf():
     o, lse = run_decode(w)
     assert np.all(o[0] == 0) and np.all(o[2] == 0)
     assert np.all(np.isneginf(lse[0])) and np.all(np.isneginf(lse[2]))
+
+
+@pytest.mark.parametrize("lengths,Hq,Hkv,D", [
+    ([3000, 1500, 700, 4096], 32, 8, 128),
+    ([2000, 300, 5000], 8, 8, 64),
+])
+def test_running_output_rescaled(lengths, Hq, Hkv, D):
+    # Keys that grow along each stream make later 16-key blocks of a chunk raise many heads' maximum
+    # score by more than 8 (base 2), which is when the split kernel rescales its running (l, o).
+    w = W.rising_decode(len(lengths), Hq, Hkv, D, lengths, seed=len(lengths) + D)
+    qn, kn, off = np64(w.q), np64(w.k), w.offsets.numpy()
+    G = Hq // Hkv
+    moved = []
+    for n, L in enumerate(lengths):
+        C = attn.default_splits(L, 16)
+        chunk = -(-L // C)
+        for c in range(C):
+            s0, s1 = int(off[n]) + c * chunk, int(off[n]) + min(L, (c + 1) * chunk)
+            if s1 <= s0:
+                continue
+            x = np.stack([w.scale * kn[s0:s1, h // G] @ qn[n, h] for h in range(Hq)])
+            moved.append(running_max_moves(x, 16) > 0)
+    moved = np.concatenate(moved)
+    assert moved.mean() > 0.25 and (~moved).mean() > 0.05, moved.mean()
+    o, lse = run_decode(w)
+    o_ref, lse_ref = ref(w)
+    assert_o_bf16(o, o_ref)
+    assert_lse(lse, lse_ref)
+
+
+# ---------------------------------------------------------------------------------------------
+# Several query tokens per stream (attn_decode_splitkv_qlen): token t of a stream with L keys sees
+# keys 0 .. L - q_len + t.
+# ---------------------------------------------------------------------------------------------
+
+def ref_qlen(w):
+    return oracle.decode_attention_qlen(np64(w.q), np64(w.k), np64(w.v), w.offsets.numpy(), w.scale)
+
+
+@pytest.mark.parametrize("lengths,q_len,Hq,Hkv,D", [
+    ([1000, 2, 513, 0, 64], 2, 32, 8, 128),     # 4 heads x 2 tokens per item (8 of 16 rows)
+    ([700, 3000, 5, 4096], 4, 32, 8, 128),      # 4 heads x 4 tokens (16 rows)
+    ([300, 1, 2048], 3, 8, 8, 64),              # one head x 3 tokens (the 4-row variant)
+    ([1500, 17, 800], 8, 8, 2, 128),            # two token passes per head group
+    ([900, 33], 16, 6, 3, 64),                  # 2 heads x 8 tokens, two passes
+    ([4096, 2000], 5, 16, 1, 128),              # G = 16: four head passes, a partial token pass
+    ([50, 10, 0], 20, 4, 4, 64),                # more tokens than 16 rows; L < q_len for one stream
+])
+def test_decode_qlen(lengths, q_len, Hq, Hkv, D):
+    w = W.random_decode(len(lengths), Hq, Hkv, D, lengths, seed=sum(lengths) + q_len, q_len=q_len)
+    o, lse = run_decode(w)
+    assert attn.last_path(2) == "decode_splitkv_qlen_mma16816"
+    assert o.shape == (len(lengths), q_len, Hq, D) and lse.shape == (len(lengths), Hq, q_len)
+    o_ref, lse_ref = ref_qlen(w)
+    assert_o_bf16(o, o_ref)
+    assert_lse(lse, lse_ref)
+
+
+def test_decode_qlen_rising_keys_and_split_counts():
+    # rows that rescale their running output, cut into different numbers of chunks
+    w = W.rising_decode(4, 32, 8, 128, [3000, 1500, 700, 4096], seed=7, q_len=4)
+    o_ref, lse_ref = ref_qlen(w)
+    for ns in (None, [1, 3, 16, 64]):
+        o, lse = run_decode(w, num_splits=ns, max_splits=64 if ns else 16)
+        assert_o_bf16(o, o_ref)
+        assert_lse(lse, lse_ref)
+
+
+def test_decode_qlen_one_token_equals_decode():
+    w3 = W.random_decode(5, 32, 8, 128, [100, 2000, 0, 1, 4096], seed=8)
+    w4 = W.random_decode(5, 32, 8, 128, [100, 2000, 0, 1, 4096], seed=8, q_len=1)
+    o3, l3 = run_decode(w3)
+    o4, l4 = run_decode(w4)
+    assert np.array_equal(o3, o4[:, 0]) and np.array_equal(l3, l4[..., 0])
+
+
+def test_decode_qlen_paged():
+    w = W.random_decode(5, 32, 8, 128, [1000, 3, 64, 4096, 77], seed=9, q_len=4)
+    o, lse, pc = run_paged(w, 64, seed=2)
+    assert attn.device_status() == 0
+    assert attn.last_path(2) == "decode_splitkv_paged_qlen_mma16816"
+    assert np.all(np.isfinite(o))
+    o_ref, lse_ref = oracle.decode_attention_paged_qlen(np64(w.q), np64(pc.k_pages), np64(pc.v_pages),
+                                                        pc.block_table.numpy(), pc.seq_lens.numpy(), w.scale)
+    assert_o_bf16(o, o_ref)
+    assert_lse(lse, lse_ref)
 
 
 # ---------------------------------------------------------------------------------------------

@@ -8,7 +8,7 @@ import torch
 import online_softmax_attention_fwd_b200 as attn
 import oracle
 from online_softmax_attention_fwd_b200 import workloads as W
-from tests._util import assert_f32, assert_lse, assert_o_bf16, np64
+from tests._util import assert_f32, assert_lse, assert_o_bf16, assert_o_fp8, np64, running_max_moves
 
 pytestmark = pytest.mark.gpu
 
@@ -124,3 +124,63 @@ def test_long_prefill_44k_sampled_rows():
     assert_lse(np.concatenate(got_l), np.concatenate(ref_l))
     # property at full size: every row is a convex combination of V rows, so |O| <= max |V|
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+
+
+@pytest.mark.parametrize("B,Sq,Sk,Hq,Hkv,D,causal", [
+    (1, 640, 640, 4, 2, 128, True),      # head pairs, five key blocks
+    (1, 600, 600, 3, 1, 64, True),       # row pairs (odd group size), ragged tail
+    (2, 384, 700, 2, 2, 128, False),     # Sq < Sk, ragged last block
+    (1, 512, 512, 8, 1, 64, False),
+    (1, 300, 900, 4, 1, 128, True),      # bottom-right causal with Sq < Sk
+])
+def test_running_output_rescaled(B, Sq, Sk, Hq, Hkv, D, causal):
+    # Keys that grow along the sequence make later key blocks raise many rows' maximum score by more
+    # than 8 (base 2) over every earlier block's, which is when the kernel multiplies the running
+    # output O in tensor memory by 2^(m_old - m_new): the monoid's rescale step. Counted here on
+    # the oracle's scores: a large share of rows must move their maximum after the first block.
+    w = W.rising_prefill(B, Sq, Sk, Hq, Hkv, D, causal, seed=Sq + Sk + D)
+    x = oracle.attention_scores(np64(w.q), np64(w.k), causal, w.scale)
+    moves = running_max_moves(x, 128)
+    assert (moves > 0).mean() > 0.25 and (moves == 0).mean() > 0.05, (moves > 0).mean()
+    check_fwd(w)
+
+
+# ---------------------------------------------------------------------------------------------
+# FP8 (e4m3) inputs with per-tensor scales (attn_fwd_fp8)
+# ---------------------------------------------------------------------------------------------
+
+def run_fp8(w):
+    dev = torch.device("cuda")
+    q, k, v = (t.to(dev) for t in (w.q, w.k, w.v))
+    o, lse = attn.fwd_fp8(q, k, v, w.q_scale, w.k_scale, w.v_scale, causal=w.causal, scale=w.scale)
+    torch.cuda.synchronize()
+    assert attn.device_status() == 0
+    assert attn.last_path(0) == "fwd_sm100_tcgen05_fp8"
+    return np64(o), np64(lse)
+
+
+def check_fp8(w):
+    o, lse = run_fp8(w)
+    o_ref, lse_ref = oracle.attention_fwd_fp8(w.q.numpy(), w.k.numpy(), w.v.numpy(), w.q_scale, w.k_scale,
+                                              w.v_scale, w.causal, w.scale)
+    assert_o_fp8(o, o_ref)
+    assert_lse(lse, lse_ref)
+
+
+@pytest.mark.parametrize("B,Sq,Sk,Hq,Hkv,causal", [
+    (1, 512, 512, 4, 2, True),       # head pairs
+    (2, 300, 300, 8, 8, False),      # ragged tail
+    (1, 1000, 1000, 3, 1, True),     # odd group size (row pairs)
+    (1, 130, 517, 8, 2, True),       # Sq < Sk
+    (1, 4096, 4096, 32, 8, True),    # the 4k GQA prefill's shape
+])
+def test_fp8_forward(B, Sq, Sk, Hq, Hkv, causal):
+    check_fp8(W.fp8_prefill(B, Sq, Sk, Hq, Hkv, 128, causal, seed=Sq + Sk))
+
+
+def test_fp8_forward_rescales_running_output():
+    w = W.fp8_prefill(1, 640, 640, 4, 2, 128, True, seed=5, rising=True)
+    x = oracle.attention_scores(w.q_scale * oracle.e4m3_to_float(w.q.numpy()),
+                                w.k_scale * oracle.e4m3_to_float(w.k.numpy()), True, w.scale)
+    assert (running_max_moves(x, 128) > 0).mean() > 0.25
+    check_fp8(w)

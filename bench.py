@@ -13,13 +13,18 @@ against the bf16 tensor peak, decode in KV GB/s against HBM bandwidth). The 4403
 prefill forward and the sequence-512 transformer-block attention are measured as extra components.
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on the launch stream;
-L2 is flushed between steps (a 512 MiB device write outside the events). Multi-GPU: one process
-per GPU (torchrun), every rank runs the same replica workload (weak scaling; no data-path
-collective), the time is the max over ranks (an all-reduce of the timing scalar only).
+L2 is flushed between steps (a 512 MiB device write outside the events). The step time is the
+median of the K steps (the mean is reported beside it). Nothing else is recorded inside that loop:
+the per-kernel split (`kernels`, `roofline`) comes from a second, separate pass with CUDA events
+around every launch. Multi-GPU: one process per GPU, every rank runs the same replica workload
+(weak scaling; no data-path collective), the time is the max over ranks (an all-reduce of the
+timing scalar only). `python bench.py --gpus N` without a process group starts the N ranks itself
+(torchrun, rendezvous on 127.0.0.1); under an existing group --gpus must equal its size.
 
 `--impl reference` times the fp64 CPU oracle (the only other implementation of this path) on a
-bounded sample of the same workload and reports the same metric, extrapolated by head and stream
-count; under torchrun only rank 0 does so.
+bounded sample of the same workload (one query head of the prefill, two decode streams) and reports
+the same metric over the sample's own work and measured seconds; the extrapolation to a whole step
+is a labelled extra field. Under torchrun only rank 0 runs it.
 """
 from __future__ import annotations
 
@@ -45,6 +50,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 CSRC = os.path.join(ROOT, "online_softmax_attention_fwd_b200", "csrc")
 # kernel family -> source file whose contents identify the kernel revision (for ncu traffic)
 KERNEL_SOURCES = {"fwd_sm100": "fwd_sm100.cu", "bwd_sm100": "bwd_sm100.cu", "decode_split": "decode.cu",
+                  "merge": "merge.cu", "fwd_sm100_fp8": "fwd_sm100.cu", "bwd_dkv_convert": "bwd_sm100.cu",
                   "decode_combine": "decode.cu", "bwd_simt_dq": "simt.cu", "bwd_simt_dkdv": "simt.cu",
                   "bwd_simt_delta": "simt.cu", "bwd_prep": "bwd_sm100.cu", "bwd_dq_convert": "bwd_sm100.cu"}
 
@@ -270,6 +276,13 @@ def oracle_sample(prefill, dec, n_heads: int, n_streams: int):
 # main benchmark
 # ------------------------------------------------------------------------------------------------
 
+def oracle_sample_flops(prefill, dec, n_heads: int, n_streams: int) -> float:
+    """Algorithmic FLOPs of the work ``oracle_sample`` does (same convention as the GPU step)."""
+    B, Sq, Hq, D = prefill.q.shape
+    f = 3.5 * prefill_fwd_flops(B, n_heads, Sq, prefill.k.shape[1], D, prefill.causal)
+    return f + decode_flops(dec.meta["lengths"][:n_streams], 1, D) * Hq
+
+
 def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
@@ -279,24 +292,27 @@ def run_reference(args):
     torch.set_num_threads(os.cpu_count() or 1)
     pre = W.gqa_prefill_4k("A")
     dec = W.decode48()
-    step_flops = 3.5 * prefill_fwd_flops(1, 32, 4096, 4096, 128, True) + decode_flops(dec.meta["lengths"], 32, 128)
+    n_heads, n_streams = 1, 2
+    sample_flops = oracle_sample_flops(pre, dec, n_heads, n_streams)
     for _ in range(args.warmup):
-        oracle_sample(pre, dec, 1, 2)
+        oracle_sample(pre, dec, n_heads, n_streams)
     secs, extrap = [], []
+    cores = 1
     for _ in range(args.steps):
-        s, e, cores = oracle_sample(pre, dec, 1, 2)
+        s, e, cores = oracle_sample(pre, dec, n_heads, n_streams)
         secs.append(s)
         extrap.append(e)
-    t = statistics.mean(extrap)
-    value = step_flops / t / 1e12
+    t = statistics.median(secs)
+    value = sample_flops / t / 1e12
     sample = ("per step: fp64 oracle forward+backward on 1 of 32 query heads of the 4k GQA prefill and "
-              "decode of 2 of 48 streams, extrapolated by head count and cached-key count")
+              "decode of 2 of 48 streams; value = that sample's algorithmic FLOPs / its measured seconds")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_block(),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                             "sample": sample, "sample_seconds_per_step": statistics.mean(secs)},
+                             "sample": sample, "sample_seconds_per_step": t,
+                             "extrapolated_full_step_seconds": statistics.median(extrap)},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -364,7 +380,8 @@ def run_ours(args):
         step()
     torch.cuda.synchronize()
 
-    # ---------------- timed region: K steps, per-step events, L2 flushed between steps
+    # ---------------- timed region: K steps, per-step events, L2 flushed between steps (the flush
+    # runs outside the events); no per-launch profiling events inside this loop
     sampler = ClockSampler(local)
     sampler.start()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
@@ -372,7 +389,6 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize()
     launches0 = attn.launch_count()
-    attn.profile_start()
     t_wall0 = time.perf_counter()
     for i in range(args.steps):
         flush.zero_()
@@ -381,16 +397,28 @@ def run_ours(args):
         evs[i][1].record(stream)
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall0
-    prof = attn.profile_stop()
     launches = attn.launch_count() - launches0
     if ws > 1:
         dist.barrier()
     clocks = sampler.stop()
     step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_s = sum(step_ms) / 1e3
-    max_total_s = reduce_max(total_s, dev)
-    value = whole_job_rate(step_flops, args.steps, ws, max_total_s) / 1e12
+    med_s = reduce_max(statistics.median(step_ms) / 1e3, dev)
+    mean_s = reduce_max(statistics.mean(step_ms) / 1e3, dev)
+    value = whole_job_rate(step_flops, 1, ws, med_s) / 1e12
     status = attn.device_status()
+
+    # ---------------- per-kernel split: a second, separate pass with CUDA events around every launch
+    prof_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    attn.profile_start()
+    for _ in range(prof_steps):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    prof = attn.profile_stop()
 
     # ---------------- per-part timing (each part alone, same hygiene) for the components
     def time_part(fn, iters):
@@ -437,6 +465,57 @@ def run_ours(args):
         components["decode48_paged64"] = {"ms": t_pg * 1e3, "kv_gbs": b_dec / t_pg / 1e9,
                                           "frac_of_hbm": b_dec / t_pg / 1e9 / peaks["hbm_gbs"]}
         del kp, vp, bt, sl, pc
+        # the same 48 streams with four query tokens each (a speculative step): same keys read once
+        wq = W.random_decode(48, 32, 8, 128, lengths.tolist(), seed=0, q_len=4)
+        qd4 = wq.q.to(dev)
+        od4 = torch.empty_like(qd4)
+        l4 = torch.empty(48, 32, 4, dtype=torch.float32, device=dev)
+        ws4 = torch.empty(attn.decode_workspace_size(48 * 4, Hq, D, 16), dtype=torch.uint8, device=dev)
+        t_d4 = time_part(lambda: attn.decode(qd4, kd, vd, off, max_splits=16, scale=dec.scale, out=od4, lse=l4,
+                                             workspace=ws4), iters)
+        b_d4 = decode_bytes(lengths, Hq * 4, Hkv, D)
+        components["decode48_qlen4"] = {"ms": t_d4 * 1e3, "kv_gbs": b_d4 / t_d4 / 1e9,
+                                        "frac_of_hbm": b_d4 / t_d4 / 1e9 / peaks["hbm_gbs"],
+                                        "tflops": 4 * f_dec / t_d4 / 1e12}
+        del qd4, od4, l4, ws4
+        # packed variable-length prefill: 8 causal prompts of 512-4096 tokens, forward and backward
+        wv = W.varlen_prefill_8x()
+        qv, kv_, vv, dov, cqv, ckv = (t.to(dev) for t in (wv.q, wv.k, wv.v, wv.do, wv.cu_q, wv.cu_k))
+        lv = wv.meta["lengths_q"].tolist()
+        mv = max(lv)
+        fv = sum(prefill_fwd_flops(1, 32, L, L, 128, True) for L in lv)
+        ov, lsev = attn.fwd_varlen(qv, kv_, vv, cqv, ckv, mv, mv, causal=True, scale=wv.scale)
+        wsv = torch.empty(attn.lib().attn_bwd_varlen_workspace_size(8, 32, 8, mv, mv, 128), dtype=torch.uint8, device=dev)
+        gv = tuple(torch.empty_like(t) for t in (qv, kv_, vv))
+        t_vf = time_part(lambda: attn.fwd_varlen(qv, kv_, vv, cqv, ckv, mv, mv, causal=True, scale=wv.scale,
+                                                 out=ov, lse=lsev), iters)
+        t_vb = time_part(lambda: attn.bwd_varlen(qv, kv_, vv, ov, lsev, dov, cqv, ckv, mv, mv, causal=True,
+                                                 scale=wv.scale, workspace=wsv, out=gv), iters)
+        components["varlen8x_fwd"] = {"ms": t_vf * 1e3, "tflops": fv / t_vf / 1e12,
+                                      "frac_of_bf16_peak": fv / t_vf / 1e12 / peaks["bf16_tflops"],
+                                      "tokens": sum(lv)}
+        components["varlen8x_bwd"] = {"ms": t_vb * 1e3, "tflops": 2.5 * fv / t_vb / 1e12,
+                                      "frac_of_bf16_peak": 2.5 * fv / t_vb / 1e12 / peaks["bf16_tflops"]}
+        del qv, kv_, vv, dov, ov, lsev, wsv, gv
+        # FP8 (e4m3) forward at the 4k GQA shape, against the fp8 dense peak (2x the measured bf16)
+        w8 = W.fp8_prefill(1, 4096, 4096, 32, 8, 128, True, seed=0)
+        q8, k8, v8 = (t.to(dev) for t in (w8.q, w8.k, w8.v))
+        o8, l8 = attn.fwd_fp8(q8, k8, v8, w8.q_scale, w8.k_scale, w8.v_scale, causal=True, scale=w8.scale)
+        t8 = time_part(lambda: attn.fwd_fp8(q8, k8, v8, w8.q_scale, w8.k_scale, w8.v_scale, causal=True,
+                                            scale=w8.scale, out=o8, lse=l8), iters)
+        components["fp8_gqa4k_fwd"] = {"ms": t8 * 1e3, "tflops": f_fwd / t8 / 1e12,
+                                       "frac_of_fp8_peak": f_fwd / t8 / 1e12 / (2.0 * peaks["bf16_tflops"]),
+                                       "fp8_peak_note": "2 x measured bf16 (nominal fp8 / bf16 dense ratio 4.5 / 2.25)"}
+        del q8, k8, v8, o8, l8
+        # monoid merge of two partial attentions of the 4k prefill's shape (a context-parallel step)
+        o_acc = torch.zeros(B, Sq, Hq, D, dtype=torch.float32, device=dev)
+        l_acc = torch.zeros(B, Hq, Sq, dtype=torch.float32, device=dev)
+        o_mo = torch.empty_like(o)
+        t_m = time_part(lambda: attn.merge(o_acc, l_acc, o, lse, o_mo), iters)
+        b_m = B * Sq * Hq * D * (4 + 4 + 2 + 2) + B * Hq * Sq * 4 * 3
+        components["merge_gqa4k"] = {"ms": t_m * 1e3, "gbs": b_m / t_m / 1e9,
+                                     "frac_of_hbm": b_m / t_m / 1e9 / peaks["hbm_gbs"]}
+        del o_acc, l_acc, o_mo
         w5 = W.long_prefill_44k()
         q5, k5, v5 = (t.to(dev) for t in (w5.q, w5.k, w5.v))
         o5, l5 = attn.fwd(q5, k5, v5, causal=True, scale=w5.scale)
@@ -447,7 +526,7 @@ def run_ours(args):
         del q5, k5, v5, o5, l5
 
     # ---------------- roofline of the dominant kernel (live CUDA events around each launch)
-    work = {"fwd_sm100": ("tensor", f_fwd), "bwd_sm100": ("tensor", f_bwd),
+    work = {"fwd_sm100": ("tensor", f_fwd), "bwd_sm100": ("tensor", f_bwd), "merge": ("hbm", None),
             "bwd_simt_dq": ("alu", None), "bwd_simt_dkdv": ("alu", None),
             "decode_split": ("hbm", b_dec), "decode_combine": ("hbm", None)}
     roofline = roofline_entry(prof, work, peaks, peak_src)
@@ -489,13 +568,15 @@ def run_ours(args):
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": max_total_s / args.steps * 1e3, "higher_is_better": True,
+                "warmup": args.warmup, "ms_per_step": med_s * 1e3, "ms_per_step_mean": mean_s * 1e3,
+                "step_statistic": "median over the K timed steps, max over ranks", "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": config_block(), "clocks": clocks,
                 "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h, "ms_per_step": e2e_s * 1e3},
                 "gpu_launches": launches, "roofline": roofline, "cpu_baseline": cpu,
                 "components": components, "kernels": kernels,
+                "kernels_note": f"per-kernel CUDA events from a separate {prof_steps}-step pass after the timed region",
                 "wall_s_timed_region": t_wall, "device_status": status,
                 "peaks": {**peaks, "source": peak_src}}
         print(json.dumps(line), flush=True)
@@ -508,6 +589,9 @@ def run_ours(args):
 def run_case(name):
     """One launch of each kernel of a workload and nothing else (a small command for ncu captures):
     `prefill` = the 4k GQA causal forward and backward, `decode` = the 48-stream split-KV decode,
+    `decode_paged` = the same 48 streams read from a cache of 64-key pages, `decode_qlen` = the 48
+    streams with four query tokens each, `varlen` = the packed 8-prompt prefill forward and backward,
+    `fp8` = the FP8 forward at the 4k GQA shape,
     `long` = the forward of the long-prefill workload at S = 16384 (the 44k workload's construction
     and kernel at a size that a full ncu capture handles; about 0.4 GB on the device)."""
     import torch
@@ -523,6 +607,26 @@ def run_case(name):
         q, k, v, do = (t.to(dev) for t in (w.q, w.k, w.v, w.do))
         o, lse = attn.fwd(q, k, v, causal=True, scale=w.scale)
         attn.bwd(q, k, v, o, lse, do, causal=True, scale=w.scale)
+    elif name == "decode_qlen":
+        wd = W.decode48()
+        wq = W.random_decode(48, 32, 8, 128, wd.meta["lengths"].tolist(), seed=0, q_len=4)
+        q, k, v, off = (t.to(dev) for t in (wq.q, wd.k, wd.v, wd.offsets))
+        attn.decode(q, k, v, off, scale=wd.scale)
+    elif name == "varlen":
+        w = W.varlen_prefill_8x()
+        q, k, v, do, cq, ck = (t.to(dev) for t in (w.q, w.k, w.v, w.do, w.cu_q, w.cu_k))
+        m = int(w.meta["lengths_q"].max())
+        o, lse = attn.fwd_varlen(q, k, v, cq, ck, m, m, causal=True, scale=w.scale)
+        attn.bwd_varlen(q, k, v, o, lse, do, cq, ck, m, m, causal=True, scale=w.scale)
+    elif name == "fp8":
+        w = W.fp8_prefill(1, 4096, 4096, 32, 8, 128, True, seed=0)
+        q, k, v = (t.to(dev) for t in (w.q, w.k, w.v))
+        attn.fwd_fp8(q, k, v, w.q_scale, w.k_scale, w.v_scale, causal=True, scale=w.scale)
+    elif name == "decode_paged":
+        wd = W.decode48()
+        pc = W.paged_from_packed(wd, 64, seed=0)
+        q, kp, vp, bt, sl = (t.to(dev) for t in (wd.q, pc.k_pages, pc.v_pages, pc.block_table, pc.seq_lens))
+        attn.decode_paged(q, kp, vp, bt, sl, scale=wd.scale)
     else:
         wd = W.decode48()
         q, k, v, off = (t.to(dev) for t in (wd.q, wd.k, wd.v, wd.offsets))
@@ -533,6 +637,23 @@ def run_case(name):
     return 0 if status == 0 else 1
 
 
+def launch_ranks(n: int, script: str, argv, port: int = 0, timeout_s: float = 1800.0) -> int:
+    """Runs ``script argv`` as ``n`` ranks of one node under torchrun (rendezvous on 127.0.0.1),
+    passing through what the ranks print; returns torchrun's exit code. ``bench.py --gpus N`` uses it
+    when it is started without a process group (no WORLD_SIZE in the environment)."""
+    if port == 0:
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", script] + list(argv)
+    r = subprocess.run(cmd, stdout=subprocess.PIPE, stderr=sys.stderr, text=True, timeout=timeout_s)
+    sys.stdout.write(r.stdout)
+    sys.stdout.flush()
+    return r.returncode
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -541,13 +662,21 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true")
-    ap.add_argument("--case", choices=["prefill", "decode", "long"],
+    ap.add_argument("--case", choices=["prefill", "decode", "long", "decode_paged", "decode_qlen", "varlen", "fp8"],
                     help="run one launch of each kernel of this workload and exit (for profilers)")
     args = ap.parse_args()
     if args.case:
         return run_case(args.case)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    ws = int(os.environ.get("WORLD_SIZE", "0"))
+    if ws == 0 and args.gpus > 1:
+        # no process group yet: start one rank per GPU and let them run this same command
+        return launch_ranks(args.gpus, os.path.abspath(__file__), sys.argv[1:])
+    if ws and ws != args.gpus:
+        ap.error(f"--gpus {args.gpus} does not match the {ws} ranks of this process group")
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

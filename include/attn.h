@@ -71,6 +71,19 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
                        int B, int Hq, int Hkv, int Sq, int Sk, int D, int causal, float scale,
                        attn_stream_t stream);
 
+/* attn_fwd_fp8: FP8 (e4m3) inputs with per-tensor scales (the FP8 checkpoint that the third
+ *   paragraph of "Aprofundamento" credits with a far shorter time to first token). q [B,Sq,Hq,D],
+ *   k / v [B,Sk,Hkv,D] hold E4M3 codes (one byte each: sign, 4 exponent bits with bias 7, 3 mantissa
+ *   bits; S.1111.111 is NaN); the real inputs are q_scale * q, k_scale * k, v_scale * v (scales > 0,
+ *   finite). Scores and P V run on the tensor cores as kind::f8f6f4 with fp32 accumulation; P is
+ *   rounded to e4m3 before P V (its largest value is 2^8 under the kernel's lazy rescale, within
+ *   e4m3's range), so O is accurate to e4m3's precision, not bf16's. o [B,Sq,Hq,D] bf16, lse
+ *   [B,Hq,Sq] fp32 as for attn_fwd. D must be 128 (else ATTN_ERR_UNSUPPORTED). */
+attn_status_t attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                           float q_scale, float k_scale, float v_scale,
+                           int B, int Hq, int Hkv, int Sq, int Sk, int D, int causal, float scale,
+                           attn_stream_t stream);
+
 attn_status_t attn_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
                            int B, int Hq, int Hkv, int Sq, int Sk, int D, int causal, float scale,
                            attn_stream_t stream);
@@ -108,6 +121,44 @@ attn_status_t attn_bwd_f32(const float* q, const float* k, const float* v, const
                            attn_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------ *
+ * Packed variable-length prefill.  (The multi-stream prefill behind the 44k-token time to first
+ * token of "Não escreva kernels, derive-os", "Aprofundamento", third paragraph: a serving engine
+ * prefills several prompts of different lengths at once, packed back to back without padding.)
+ *
+ * Sequence b (0 <= b < B) owns query rows cu_seqlens_q[b] .. cu_seqlens_q[b+1] - 1 of q / o / dout /
+ * dq and key/value rows cu_seqlens_k[b] .. cu_seqlens_k[b+1] - 1 of k / v / dk / dv, and attends only
+ * to its own keys, with the same definition as attn_fwd / attn_bwd per sequence (causal: bottom-right
+ * aligned within the sequence). A sequence with no key gives its rows O = 0, lse = -inf and zero
+ * gradients.
+ *   q, o, dout, dq [total_q, Hq, D] bf16; k, v, dk, dv [total_k, Hkv, D] bf16; lse [Hq, total_q] fp32.
+ *   cu_seqlens_q / cu_seqlens_k: [B+1] int32 DEVICE arrays (4-byte aligned), non-decreasing, first
+ *   entry 0, last entry total_q / total_k. max_seqlen_q / max_seqlen_k: upper bounds of the sequence
+ *   lengths (they size the grids and the backward's workspace). The offsets live on the device and
+ *   are checked there: a sequence whose rows fall outside [0, total) or exceed the max_seqlen bound
+ *   is not read or written (its outputs are left as they were) and the device status records
+ *   ATTN_ERR_INVALID_ARG (attn_get_device_status).
+ *   Tiles of one sequence may read rows of the next one in the packed tensors (their keys are masked,
+ *   their values weighted by 0, their query rows not stored), so those rows must hold finite values.
+ *   D is 64 or 128. The backward's workspace: attn_bwd_varlen_workspace_size(B, Hq, Hkv,
+ *   max_seqlen_q, max_seqlen_k, D) bytes, 256-byte aligned (fp32 dQ accumulator and per-row
+ *   statistics, max_seqlen_q rows per sequence and head, and fp32 dK / dV room for the key tiles the
+ *   kernel splits over two CTAs).
+ * ------------------------------------------------------------------------------------------ */
+attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                              const int* cu_seqlens_q, const int* cu_seqlens_k, int B,
+                              int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                              int Hq, int Hkv, int D, int causal, float scale, attn_stream_t stream);
+
+size_t attn_bwd_varlen_workspace_size(int B, int Hq, int Hkv, int max_seqlen_q, int max_seqlen_k, int D);
+
+attn_status_t attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                              const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                              const int* cu_seqlens_q, const int* cu_seqlens_k, int B,
+                              int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                              int Hq, int Hkv, int D, int causal, float scale,
+                              void* workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------ *
  * Split-KV decode.  (Decode streams of "Não escreva kernels, derive-os", "Aprofundamento", third
  * paragraph; the aibriefing page, "Details", ties its 48-stream accuracy to split granularity.)
  *
@@ -143,8 +194,10 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k, const void* v,
  * library holds until the process exits. Problems needing more than 16 MiB of partial triples
  * (attn_decode_workspace_size(N, Hq, D, max_splits) > 16777216) return ATTN_ERR_WORKSPACE before
  * anything is launched; e.g. 48 streams x 32 heads x 16 splits at D = 128 need 12.8 MB and fit.
- * The first call on each device looks up the array's device address (once per device, with that
- * device current); make that first call before any stream capture. All calls share the array and
+ * The first call on each device looks up the array's device address (with that device current)
+ * and keeps it for that device's current CUDA context; after the context has been torn down and
+ * created again (cudaDeviceReset), the next call looks it up again, since the library's module may
+ * then sit elsewhere. Make each such first call before any stream capture. All calls share the array and
  * leave their partial triples in it; nothing has to start at zero. Calls that overlap on the GPU
  * (other streams or threads) race on the array and give wrong results: serialise them. */
 attn_status_t attn_decode_splitkv_static(const void* q, const void* k, const void* v,
@@ -176,6 +229,58 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* 
                                 int num_pages, const int* num_splits, int max_splits, void* o, float* lse,
                                 int N, int Hq, int Hkv, int D, float scale, void* workspace,
                                 size_t workspace_bytes, attn_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------ *
+ * Decode with several query tokens per stream (speculative or chunked decode steps). The decode
+ * steps of "Não escreva kernels, derive-os" ("Aprofundamento", third paragraph) serve 16 to 48
+ * streams; a step that verifies draft tokens, or feeds a short chunk of a prompt, brings q_len new
+ * tokens per stream instead of one. Their keys and values are already the newest q_len rows of the
+ * stream's cache, so token t (0-based) sits at position L_n - q_len + t and attends to keys
+ * 0 .. L_n - q_len + t: the causal mask among the new tokens, aligned to the newest position
+ * (bottom-right, as in attn_fwd with Sq = q_len, Sk = L_n). A token that sees no key (L_n < q_len)
+ * gets O = 0 and lse = -inf. Same split + combine and the same monoid as attn_decode_splitkv; with
+ * q_len = 1 the result is that of attn_decode_splitkv.
+ *
+ *   q, o [N, q_len, Hq, D] bf16 (row (n, t, h) of o is the output of token t of stream n, head h);
+ *   lse [N, Hq, q_len] fp32 (may be NULL); q_len >= 1, N * q_len * Hq < 2^31.
+ *   k, v, kv_offsets, num_splits, max_splits, scale: as for attn_decode_splitkv (one split count per
+ *   stream, shared by its tokens).
+ *   workspace: at least attn_decode_workspace_size(N * q_len, Hq, D, max_splits) bytes, 256-byte
+ *   aligned.
+ * attn_decode_paged_qlen: the same over a paged cache (arguments as attn_decode_paged).
+ * ------------------------------------------------------------------------------------------ */
+attn_status_t attn_decode_splitkv_qlen(const void* q, const void* k, const void* v,
+                                       const int* kv_offsets, const int* num_splits, int max_splits,
+                                       void* o, float* lse, int N, int q_len, int Hq, int Hkv, int D,
+                                       float scale, void* workspace, size_t workspace_bytes,
+                                       attn_stream_t stream);
+
+attn_status_t attn_decode_paged_qlen(const void* q, const void* k_pages, const void* v_pages,
+                                     const int* block_table, int max_pages, const int* seq_lens,
+                                     int page_size, int num_pages, const int* num_splits, int max_splits,
+                                     void* o, float* lse, int N, int q_len, int Hq, int Hkv, int D,
+                                     float scale, void* workspace, size_t workspace_bytes,
+                                     attn_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------ *
+ * Merge of partial attentions.  ("Não escreva kernels, derive-os", "Aprofundamento", first
+ * paragraph: the online softmax is a monoid, so attention over a union of key sets is the merge of
+ * the attentions over each set, in any order.) A context-parallel forward across GPUs computes, on
+ * each rank, the attention of its query rows against one key/value shard after another and folds
+ * each partial result in with this call.
+ *
+ * With M = max(lse_acc, lse_part), w_a = e^(lse_acc - M), w_b = e^(lse_part - M):
+ *   lse_acc <- M + ln(w_a + w_b),   o_acc <- (w_a o_acc + w_b o_part) / (w_a + w_b),
+ * row by row; lse = -inf is the identity (its O is not read; a row that is -inf in both stays
+ * O = 0, lse = -inf).
+ *   o_acc [B, S, H, D] fp32 and lse_acc [B, H, S] fp32: the running result, read and written in
+ *   place (start it with lse_acc = -inf; o_acc may then hold anything).
+ *   o_part [B, S, H, D] bf16 and lse_part [B, H, S] fp32: a partial result as attn_fwd writes it.
+ *   o_out [B, S, H, D] bf16: if not NULL, also receives the merged O rounded to bf16.
+ *   D is 64 or 128; all pointers 16-byte aligned.
+ * ------------------------------------------------------------------------------------------ */
+attn_status_t attn_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                         void* o_out, int B, int S, int H, int D, attn_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------ *
  * Status and introspection.

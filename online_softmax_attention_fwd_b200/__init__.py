@@ -7,7 +7,11 @@ Scaled-dot-product attention computed as one reduction under the online-softmax 
 * ``bwd`` -- bf16 backward to dQ, dK, dV;
 * ``decode`` -- split-KV decode over packed varlen caches, partial (m, l, o) triples merged by the
   monoid in a combine kernel; ``decode_paged`` -- the same over a paged cache (block table);
-* ``fwd_f32`` / ``bwd_f32`` -- genuine fp32 CUDA-core versions.
+* ``fwd_f32`` / ``bwd_f32`` -- genuine fp32 CUDA-core versions;
+* ``fwd_fp8`` -- e4m3 inputs with per-tensor scales (kind::f8f6f4 tensor cores);
+* ``fwd_varlen`` / ``bwd_varlen`` -- packed sequences of different lengths (cu_seqlens);
+* ``merge`` -- the monoid merge of partial (O, lse) results; ``ring`` -- a context-parallel ring
+  forward across ranks built on it.
 
 The C entry points are declared in ``include/attn.h``; this package only marshals torch tensors to
 them (see ``_binding.py``). ``workloads`` draws the seeded synthetic inputs.
@@ -18,6 +22,7 @@ from ._binding import (  # noqa: F401
     SIGNATURES,
     bwd,
     bwd_f32,
+    bwd_varlen,
     bwd_workspace_size,
     decode,
     decode_paged,
@@ -26,9 +31,12 @@ from ._binding import (  # noqa: F401
     device_status,
     fwd,
     fwd_f32,
+    fwd_fp8,
+    fwd_varlen,
     last_path,
     launch_count,
     lib,
+    merge,
     profile_start,
     profile_stop,
     status_string,

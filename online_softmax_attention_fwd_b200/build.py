@@ -18,7 +18,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_PATH = os.path.join(HERE, "libattn.so")
-SOURCES = ["api.cu", "simt.cu", "decode.cu", "decode_static.cu", "fwd_sm100.cu", "bwd_sm100.cu"]
+FAULT_LIB_PATH = os.path.join(HERE, "libattn_faultinject.so")  # test-only build, see build()
+SOURCES = ["api.cu", "simt.cu", "decode.cu", "decode_static.cu", "fwd_sm100.cu", "bwd_sm100.cu", "merge.cu"]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ARCH_FLAGS + ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE,
@@ -32,7 +33,7 @@ def nvcc() -> str:
 
 def _deps():
     hdrs = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))]
-    return hdrs + [os.path.join(INCLUDE, "attn.h")]
+    return hdrs + [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
 
 
 def _stale(target: str, inputs) -> bool:
@@ -42,11 +43,13 @@ def _stale(target: str, inputs) -> bool:
     return any(os.path.getmtime(x) > t for x in inputs)
 
 
-def _compile(src: str, force: bool, ptxas_verbose: bool) -> str:
-    obj = os.path.join(BUILD_DIR, os.path.splitext(src)[0] + ".o")
+def _compile(src: str, force: bool, ptxas_verbose: bool, fault_inject: bool = False) -> str:
+    sub = os.path.join(BUILD_DIR, "faultinject") if fault_inject else BUILD_DIR
+    obj = os.path.join(sub, os.path.splitext(src)[0] + ".o")
     srcp = os.path.join(CSRC, src)
     if force or _stale(obj, [srcp] + _deps()):
-        cmd = [nvcc()] + CFLAGS + (["-Xptxas", "-v"] if ptxas_verbose else []) + ["-c", srcp, "-o", obj]
+        flags = CFLAGS + (["-DATTN_FAULT_INJECT"] if fault_inject else [])
+        cmd = [nvcc()] + flags + (["-Xptxas", "-v"] if ptxas_verbose else []) + ["-c", srcp, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
@@ -55,16 +58,25 @@ def _compile(src: str, force: bool, ptxas_verbose: bool) -> str:
     return obj
 
 
-def build(force: bool = False, ptxas_verbose: bool = False) -> str:
-    """Compile every CUDA source for sm_100a and link libattn.so; returns the library path."""
-    os.makedirs(BUILD_DIR, exist_ok=True)
-    with concurrent.futures.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, force, ptxas_verbose), SOURCES))
-    if force or _stale(LIB_PATH, objs):
-        cmd = [nvcc()] + ARCH_FLAGS + ["-shared", "-o", LIB_PATH] + objs
+def _link(objs, target: str, force: bool) -> None:
+    if force or _stale(target, objs):
+        cmd = [nvcc()] + ARCH_FLAGS + ["-shared", "-o", target] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
+
+
+def build(force: bool = False, ptxas_verbose: bool = False) -> str:
+    """Compile every CUDA source for sm_100a and link libattn.so, and the test-only
+    fault-injection build libattn_faultinject.so (the same sources with ATTN_FAULT_INJECT: short
+    wait limits and a switch that makes one producer skip one copy, for the timeout tests). Returns
+    the path of libattn.so."""
+    os.makedirs(os.path.join(BUILD_DIR, "faultinject"), exist_ok=True)
+    jobs = [(s, False) for s in SOURCES] + [(s, True) for s in SOURCES]
+    with concurrent.futures.ThreadPoolExecutor(max_workers=len(jobs)) as ex:
+        objs = list(ex.map(lambda j: _compile(j[0], force, ptxas_verbose and not j[1], j[1]), jobs))
+    _link(objs[:len(SOURCES)], LIB_PATH, force)
+    _link(objs[len(SOURCES):], FAULT_LIB_PATH, force)
     return LIB_PATH
 
 

@@ -1,7 +1,7 @@
 // common.cuh -- device primitives shared by the attention kernels (sm_100a).
 //
-// Inline-PTX wrappers for mbarriers (with bounded waits), TMA tensor loads (no cluster multicast
-// anywhere), tcgen05 tensor-memory allocation / MMA / load / store, and the shared-memory matrix
+// Inline-PTX wrappers for mbarriers (with bounded waits), TMA tensor loads (each to one CTA's
+// shared memory), tcgen05 tensor-memory allocation / MMA / load / store, and the shared-memory matrix
 // and instruction descriptors of the 5th-generation tensor cores. Written from the PTX ISA's
 // instruction forms; nothing here computes attention.
 #pragma once
@@ -19,8 +19,14 @@ constexpr int kStatusBadArg = 1;    // an index read on the device is out of ran
 constexpr int kStatusTimeout = 6;
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer (2 s): far above any
-// legitimate wait in these kernels, far below a hang.
+// legitimate wait in these kernels, far below a hang. The test-only fault-injection build
+// (ATTN_FAULT_INJECT, never the shipped library) uses 20 ms so that its tests of the timeout path
+// end quickly; its kernels only ever run small problems.
+#ifdef ATTN_FAULT_INJECT
+constexpr uint64_t kWaitLimitNs = 20000000ull;
+#else
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+#endif
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -209,7 +215,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 
 // ---------------------------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), tile mode, completion through an mbarrier's transaction count.
-// No .multicast::cluster form is used anywhere in this library.
+// Every load here has a single destination CTA: no cluster-broadcast form exists in this library.
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -338,6 +344,24 @@ __device__ __forceinline__ void umma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, u
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// The same two forms with kind::f8f6f4: 8-bit A and B (e4m3 here), K = 32 per instruction, fp32
+// accumulator. An A operand in tensor memory holds four 8-bit values per 32-bit column.
+__device__ __forceinline__ void umma_ss_warp_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_ts_warp_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void umma_commit_warp(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
@@ -409,6 +433,22 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_maj
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn_major) << 15) |
          (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor for kind::f8f6f4 with e4m3 A and B and an fp32 accumulator: D format F32
+// (bits [4,6) = 1), A and B format E4M3 (0 in [7,10) and [10,13)), majors and shape as above.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, int a_mn_major, int b_mn_major) {
+  return (1u << 4) | (static_cast<uint32_t>(a_mn_major) << 15) | (static_cast<uint32_t>(b_mn_major) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Four fp32 values to e4m3 (round to nearest even, saturating to +-448), packed with `a` in the
+// lowest byte. cvt.e4m3x2 puts its first source in the upper byte of the pair.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  uint16_t lo, hi;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
 // Byte offset of the 16-byte chunk `chunk` (0..7) of row `row` inside a 128-byte-swizzled tile

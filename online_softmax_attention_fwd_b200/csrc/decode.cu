@@ -49,7 +49,7 @@ __host__ __device__ inline int decode_split_rule(int L, int max_splits) {
 int decode_default_splits(int L, int max_splits) { return decode_split_rule(L, max_splits); }
 
 size_t decode_workspace_bytes(int N, int Hq, int D, int max_splits) {
-  const size_t slots = static_cast<size_t>(N) * Hq * max_splits;
+  const size_t slots = static_cast<size_t>(N) * Hq * max_splits;  // N counts (stream, query token) rows
   const size_t o_bytes = (slots * D * sizeof(float) + 255) & ~static_cast<size_t>(255);
   const size_t ml_bytes = (slots * 2 * sizeof(float) + 255) & ~static_cast<size_t>(255);
   return o_bytes + ml_bytes;
@@ -94,80 +94,101 @@ constexpr int kDecStages = 8;
 // With eight stages each warp owns two, so its next block is in flight while it computes one.
 static_assert(kDecStages % 4 == 0, "decode ring stages must be a multiple of the compute warps");
 constexpr int kDecThreads = 160;          // four compute warps + one producer warp
-constexpr int kDecCtasPerSm = 3;
 constexpr int kDecMapRows = 0x7fffffff;   // nominal row extent of the K/V tensor maps
 // Up to this many streams, every CTA numbers the valid items densely (a prefix sum of the per-stream
 // item counts in shared memory), so the static round-robin hands each CTA the same number of items
 // to within one; above it, CTAs walk the slot space and skip the slots past a stream's split count.
 constexpr int kDecDenseMax = 256;
 
-template <int D>
+// The query rows of one item are rows of the m16n8k16 products: row r is query token tq0 + r / GT
+// and query head h0 + r % GT. RM is the number of rows the kernel variant carries: 4 (one row per
+// lane quad, rows 4-15 zero; one query token per stream, the 48-stream decode) or 16 (two rows per
+// lane quad, for several query tokens per stream). The smaller variant fits three CTAs per SM.
+template <int RM>
+constexpr int dec_ctas_per_sm() {
+  return RM == 4 ? 3 : 2;
+}
+
+template <int D, int RM>
 struct DecCfg {
   static constexpr int kAtoms = D / 64;
   static constexpr int kAtomBytes = kDecBlk * 128;       // 16 rows x 128 bytes
   static constexpr int kBlkBytes = kAtoms * kAtomBytes;  // 16 key rows x D bf16
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kDecStages * kBlkBytes;
-  static constexpr int kOffQ = 2 * kDecStages * kBlkBytes;  // [2 items][<= 4 heads][D] bf16
-  static constexpr int kQBuf = 4 * D * 2;
-  static constexpr int kOffDep = kOffQ + 2 * kQBuf;         // warps 1-3: [3][<= 4 heads][D] fp32
-  static constexpr int kOffBar = kOffDep + 3 * 4 * D * 4;
+  static constexpr int kOffQ = 2 * kDecStages * kBlkBytes;  // [2 items][RM rows][D] bf16
+  static constexpr int kQBuf = RM * D * 2;
+  static constexpr int kOffDep = kOffQ + 2 * kQBuf;         // warps 1-3: [3][RM rows][D] fp32
+  static constexpr int kOffBar = kOffDep + 3 * RM * D * 4;
   static constexpr int kNumBars = 2 * kDecStages + 4;       // full, empty, q_full[2], q_empty[2]
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;   // abort flag, then the deposits' (m, l)
-  static constexpr int kOffBase = kOffMisc + 16 + 2 * 3 * 4 * 4;  // dense item numbering, see below
+  static constexpr int kOffBase = kOffMisc + 16 + 2 * 3 * RM * 4;  // dense item numbering, see below
   static constexpr int kSmemBytes = kOffBase + (kDecDenseMax + 1) * 4 + 1024;
+  static_assert(kSmemBytes * dec_ctas_per_sm<RM>() <= 232448, "shared memory per SM");
 };
 
-// One work item: the key chunk c of stream n for the query heads h0 .. h0 + GT - 1 of kv head g.
+// How the query rows of a stream are cut into items: q_len query tokens per stream (the newest
+// q_len positions of its cache), GT query heads and TQ query tokens per item, ntp = ceil(q_len / TQ)
+// token passes.
+struct DecQ {
+  int q_len, GT, TQ, ntp;
+  int fault_block;  // test-only fault-injection build: CTA 0 skips this ring block's copy (-1: none)
+};
+
+// One work item: the key chunk c of stream n for query heads h0 .. h0 + GT - 1 (of kv head g) and
+// query tokens tq0 .. tq0 + TQ - 1. L = the stream's length; keys k0 .. k1 - 1 of the stream; nblk
+// 16-key blocks, ending at the last key any of the item's tokens can see.
 struct DecItem {
-  int n, c, g, h0, start, k0, k1, nblk;
+  int n, c, g, h0, tq0, start, L, k0, k1, nblk;
 };
 
-// Item slot idx -> item; false for slots past the stream's split count. Slots are ordered chunk
-// index slowest, so the first chunks of every stream and kv head come first.
-// The item whose fields are (n, c, gi) -> it; L = the stream's length, C_n its split count.
+// The item whose fields are (n, c, gi) -> it; C_n is the stream's split count. Items of one chunk
+// are numbered kv head slowest, so the head and token passes that read the same keys are adjacent.
 // With `aligned`, chunks are rounded up to whole 16-key blocks (a paged cache: a block must not
 // straddle two pages); the last chunks of a stream may then be empty.
-template <int GT>
 __device__ __forceinline__ void dec_item_fill(int n, int c, int gi, int start, int L, int C_n, int Hq, int Hkv,
-                                              bool aligned, DecItem& it) {
-  const int G = Hq / Hkv, npass = G / GT;
+                                              const DecQ& dq, bool aligned, DecItem& it) {
+  const int G = Hq / Hkv, npass = G / dq.GT, per_g = npass * dq.ntp;
   int chunk = (L + C_n - 1) / C_n;
   if (aligned) chunk = (chunk + kDecBlk - 1) / kDecBlk * kDecBlk;
   it.n = n;
   it.c = c;
-  it.g = gi / npass;
-  it.h0 = it.g * G + (gi % npass) * GT;
+  it.g = gi / per_g;
+  const int r = gi - it.g * per_g;
+  it.h0 = it.g * G + (r / dq.ntp) * dq.GT;
+  it.tq0 = (r % dq.ntp) * dq.TQ;
   it.start = start;
+  it.L = L;
   it.k0 = min(L, c * chunk);
   it.k1 = min(L, it.k0 + chunk);
-  it.nblk = (it.k1 - it.k0 + kDecBlk - 1) / kDecBlk;
+  // token t sees the stream's keys 0 .. L - q_len + t (the newest q_len positions are its own)
+  const int last_tok = min(dq.q_len, it.tq0 + dq.TQ) - 1;
+  const int kend = min(it.k1, max(it.k0, L - dq.q_len + last_tok + 1));
+  it.nblk = (kend - it.k0 + kDecBlk - 1) / kDecBlk;
 }
 
 // Dense item k -> item, with base[n] = NG * (C_0 + ... + C_{n-1}) in shared memory (N + 1 entries):
-// stream n holds items base[n] .. base[n + 1] - 1, chunk c = r / NG, kv head group gi = r % NG. The
-// kv heads of one chunk are consecutive items, so neighbouring CTAs read the same cache rows at
+// stream n holds items base[n] .. base[n + 1] - 1, chunk c = r / NG, head/token group gi = r % NG.
+// The groups of one chunk are consecutive items, so neighbouring CTAs read the same cache rows at
 // about the same time (a row holds every kv head's keys side by side).
-template <int GT>
-__device__ __forceinline__ void dec_item_dense(int k, int N, int Hq, int Hkv, const DecKV& kv, const int* base,
-                                               DecItem& it) {
+__device__ __forceinline__ void dec_item_dense(int k, int N, int Hq, int Hkv, const DecKV& kv, const DecQ& dq,
+                                               const int* base, DecItem& it) {
   int lo = 0, hi = N;  // largest n with base[n] <= k
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (base[mid] <= k) lo = mid; else hi = mid;
   }
-  const int NG = Hkv * ((Hq / Hkv) / GT);
+  const int NG = Hkv * ((Hq / Hkv) / dq.GT) * dq.ntp;
   const int C_n = (base[lo + 1] - base[lo]) / NG;
   const int r = k - base[lo];
   int start, L;
   dec_stream(kv, lo, start, L);
-  dec_item_fill<GT>(lo, r / NG, r % NG, start, L, C_n, Hq, Hkv, kv.block_table != nullptr, it);
+  dec_item_fill(lo, r / NG, r % NG, start, L, C_n, Hq, Hkv, dq, kv.block_table != nullptr, it);
 }
 
-template <int GT>
-__device__ __forceinline__ bool dec_item(long long idx, int N, int Hq, int Hkv, const DecKV& kv,
+__device__ __forceinline__ bool dec_item(long long idx, int N, int Hq, int Hkv, const DecKV& kv, const DecQ& dq,
                                          const int* num_splits, int max_splits, DecItem& it) {
-  const int G = Hq / Hkv, npass = G / GT, NG = Hkv * npass;
+  const int NG = Hkv * ((Hq / Hkv) / dq.GT) * dq.ntp;
   const long long per_c = static_cast<long long>(N) * NG;
   const int c = static_cast<int>(idx / per_c);
   const int r = static_cast<int>(idx - c * per_c);
@@ -176,7 +197,7 @@ __device__ __forceinline__ bool dec_item(long long idx, int N, int Hq, int Hkv, 
   dec_stream(kv, n, start, L);
   const int C_n = stream_splits(num_splits, n, L, max_splits);
   if (c >= C_n) return false;
-  dec_item_fill<GT>(n, c, gi, start, L, C_n, Hq, Hkv, kv.block_table != nullptr, it);
+  dec_item_fill(n, c, gi, start, L, C_n, Hq, Hkv, dq, kv.block_table != nullptr, it);
   return true;
 }
 
@@ -190,32 +211,34 @@ __device__ __forceinline__ bool dec_wait_drain(uint64_t* bar, uint32_t parity) {
 // Byte offset of element d of row r in a 128-byte-swizzled block of 64-element column atoms.
 template <int D>
 __device__ __forceinline__ uint32_t dec_sw(int r, int d) {
-  return (d >> 6) * DecCfg<D>::kAtomBytes + sw128_offset(r, (d & 63) >> 3) + (d & 7) * 2;
+  constexpr int kAtomBytes = kDecBlk * 128;
+  return (d >> 6) * kAtomBytes + sw128_offset(r, (d & 63) >> 3) + (d & 7) * 2;
 }
 
-template <int D, int GT>
-__global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
+template <int D, int RM>
+__global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<RM>())
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
-                        const uint16_t* __restrict__ v, const DecKV kv, int N,
+                        const uint16_t* __restrict__ v, const DecKV kv, const DecQ dq, int N,
                         const int* __restrict__ num_splits, int max_splits, int Hq, int Hkv, float scale_log2,
                         float* __restrict__ part_o, float* __restrict__ part_ml, int* status) {
-  using C = DecCfg<D>;
+  using C = DecCfg<D, RM>;
+  constexpr int NR = RM == 16 ? 2 : 1;  // rows per lane quad: g and g + 8
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem + C::kOffK;
   uint8_t* sV = smem + C::kOffV;
   uint8_t* sQ = smem + C::kOffQ;
-  float* dep = reinterpret_cast<float*>(smem + C::kOffDep);  // [3][GT][D]
+  float* dep = reinterpret_cast<float*>(smem + C::kOffDep);  // [3][RM][D]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* empty = full + kDecStages;
   uint64_t* q_full = empty + kDecStages;  // [2]
   uint64_t* q_empty = q_full + 2;         // [2]
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc);
-  float* dep_m = reinterpret_cast<float*>(smem + C::kOffMisc + 16);  // [3][4]
-  float* dep_l = dep_m + 12;                                         // [3][4]
+  float* dep_m = reinterpret_cast<float*>(smem + C::kOffMisc + 16);  // [3][RM]
+  float* dep_l = dep_m + 3 * RM;                                      // [3][RM]
 
-  const int G = Hq / Hkv, npass = G / GT, NG = Hkv * npass;
+  const int NG = Hkv * ((Hq / Hkv) / dq.GT) * dq.ntp;
   const long long n_slots = static_cast<long long>(N) * NG * max_splits;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // dense numbering of the valid items (up to kDecDenseMax streams): warp 0 scans the per-stream
@@ -260,10 +283,10 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
   // item number i of the walk -> item; false for a sparse slot past its stream's split count
   auto next_item = [&](long long i, DecItem& it) -> bool {
     if (dense) {
-      dec_item_dense<GT>(static_cast<int>(i), N, Hq, Hkv, kv, base, it);
+      dec_item_dense(static_cast<int>(i), N, Hq, Hkv, kv, dq, base, it);
       return true;
     }
-    return dec_item<GT>(i, N, Hq, Hkv, kv, num_splits, max_splits, it);
+    return dec_item(i, N, Hq, Hkv, kv, dq, num_splits, max_splits, it);
   };
 
   if (warp == 4) {
@@ -271,18 +294,22 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
     const bool paged = kv.block_table != nullptr;
     const int T = paged ? 0 : min(kv.offsets[N], kDecMapRows);  // no box may reach past the cache
     const long long rs = static_cast<long long>(Hkv) * D;
+    const uint32_t qrow_bytes = static_cast<uint32_t>(dq.GT) * D * 2;  // one token's GT heads
     long long gb = 0;  // ring position: blocks issued so far
     int qi = 0;        // items started so far
     bool ok = true;
     for (long long idx = blockIdx.x; ok && idx < n_iter; idx += gridDim.x) {
       DecItem it;
       if (!next_item(idx, it)) continue;
-      if (lane == 0) {  // the item's GT query rows (contiguous) into query buffer qi % 2
+      if (lane == 0) {  // the item's query rows (GT contiguous heads per token) into buffer qi % 2
         ok = mbar_wait(q_empty + (qi & 1), ((qi >> 1) & 1) ^ 1, abort, status);
         if (ok) {
-          mbar_arrive_expect_tx(q_full + (qi & 1), GT * D * 2);
-          bulk_load(sQ + (qi & 1) * C::kQBuf, q + (static_cast<long long>(it.n) * Hq + it.h0) * D, GT * D * 2,
-                    q_full + (qi & 1));
+          const int ntok = min(dq.TQ, dq.q_len - it.tq0);
+          mbar_arrive_expect_tx(q_full + (qi & 1), ntok * qrow_bytes);
+          for (int t = 0; t < ntok; ++t)
+            bulk_load(sQ + (qi & 1) * C::kQBuf + t * qrow_bytes,
+                      q + ((static_cast<long long>(it.n) * dq.q_len + it.tq0 + t) * Hq + it.h0) * D, qrow_bytes,
+                      q_full + (qi & 1));
         }
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -320,6 +347,12 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
           }
           __syncwarp();
         }
+#ifdef ATTN_FAULT_INJECT
+        if (blockIdx.x == 0 && gb == dq.fault_block) {  // a compute warp's wait for it runs out
+          ++gb;
+          continue;
+        }
+#endif
         if (lane == 0) {
           mbar_arrive_expect_tx(full + s, 2u * nrows * D * 2);
           if (tile) {
@@ -352,13 +385,12 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
   }
 
   // ------------------------------------------------------------------ compute warps
-  // Lane (g, t) = (lane / 4, lane % 4) holds head g: scores of keys 2t, 2t + 1, 8 + 2t, 9 + 2t of
-  // a block and output columns 8 j + 2t, 8 j + 2t + 1 of every 8-column tile j. The GT heads are
-  // the rows of the m16n8k16 products (padded to 16 with zeros), so S^T = Q K^T takes K straight
-  // from the ring as its column operand and P V takes the probabilities straight from the score
-  // accumulators.
+  // Lane (g, t) = (lane / 4, lane % 4) holds item row g (and g + 8 when RM = 16): scores of keys 2t,
+  // 2t + 1, 8 + 2t, 9 + 2t of a block and output columns 8 j + 2t, 8 j + 2t + 1 of every 8-column
+  // tile j. The item's rows (query heads x query tokens) are the rows of the m16n8k16 products
+  // (padded to 16 with zeros), so S^T = Q K^T takes K straight from the ring as its column operand
+  // and P V takes the probabilities straight from the score accumulators.
   const int gq = lane >> 2, tq = lane & 3;
-  const bool head = gq < GT;
   constexpr int KS = D / 16;  // 16-wide steps over the head dim
   const int mi = lane >> 3, ri = lane & 7;  // ldmatrix: this lane addresses row ri of matrix mi
   long long gb = 0;  // ring position of the current item's first block
@@ -369,13 +401,28 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
     if (!next_item(idx, it)) continue;
     // this item's query rows (bf16) in shared memory; each block reads its Q fragments from there
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(q_full + (qi & 1), (qi >> 1) & 1, abort, status)) != 0;
-    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(sQ + (qi & 1) * C::kQBuf) + (head ? gq : 0) * (D / 2);
     const int qbuf = qi & 1;
     ++qi;
+    const int nrow = dq.GT * min(dq.TQ, dq.q_len - it.tq0);  // valid rows of this item
+    bool valid[NR];
+    int lim[NR];  // last visible key of the row, relative to the chunk's first key
+    const uint32_t* qrow[NR];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      const int row = gq + 8 * r;
+      valid[r] = row < nrow && row < RM;
+      lim[r] = it.L - dq.q_len + it.tq0 + row / dq.GT - it.k0;
+      qrow[r] = reinterpret_cast<const uint32_t*>(sQ + qbuf * C::kQBuf) + (valid[r] ? row : 0) * (D / 2);
+    }
     float o[D / 8][4];
 #pragma unroll
     for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-    float mrow = -INFINITY, lrow = 0.f;  // head gq: running max (base 2) and this lane's share of the sum
+    float mrow[NR], lrow[NR];  // per row: running max (base 2) and this lane's share of the sum
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      mrow[r] = -INFINITY;
+      lrow[r] = 0.f;
+    }
     for (int bk = (warp - static_cast<int>(gb & 3)) & 3; ok && bk < it.nblk; bk += 4) {
       const long long gbk = gb + bk;
       const int s = static_cast<int>(gbk % kDecStages);
@@ -384,56 +431,74 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
       if (!ok) break;
       const uint32_t kb = smem_u32(sK + s * C::kBlkBytes);
       const uint32_t vb = smem_u32(sV + s * C::kBlkBytes);
-      const int nk = min(kDecBlk, it.k1 - (it.k0 + bk * kDecBlk));
-      // S^T for keys 0-7 (s0) and 8-15 (s1)
+      const int nk = min(kDecBlk, it.k1 - (it.k0 + bk * kDecBlk));  // keys of the chunk in this block
+      // S^T for keys 0-7 (s0) and 8-15 (s1); rows g in s*[0..1], rows g + 8 in s*[2..3]
       float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
-        // Q fragments of head gq (zero for the padding rows): head dims 16 ks + 2t .. and + 8
-        const uint32_t qa = head ? qrow[8 * ks + tq] : 0u, qb = head ? qrow[8 * ks + 4 + tq] : 0u;
+        // Q fragments of the lane's rows (zero for padding rows): head dims 16 ks + 2t .. and + 8
+        const uint32_t qa = valid[0] ? qrow[0][8 * ks + tq] : 0u, qb = valid[0] ? qrow[0][8 * ks + 4 + tq] : 0u;
+        uint32_t qc = 0u, qd = 0u;
+        if (NR == 2) {
+          qc = valid[NR - 1] ? qrow[NR - 1][8 * ks + tq] : 0u;
+          qd = valid[NR - 1] ? qrow[NR - 1][8 * ks + 4 + tq] : 0u;
+        }
         uint32_t b00, b01, b10, b11;  // matrices: keys 8 (mi / 2) + ri, head dims 16 ks + 8 (mi % 2) ..
         ldsm_x4(kb + dec_sw<D>(ri + 8 * (mi >> 1), 16 * ks + 8 * (mi & 1)), b00, b01, b10, b11);
-        mma_16816(s0, qa, 0u, qb, 0u, b00, b01);
-        mma_16816(s1, qa, 0u, qb, 0u, b10, b11);
+        mma_16816(s0, qa, qc, qb, qd, b00, b01);
+        mma_16816(s1, qa, qc, qb, qd, b10, b11);
       }
-      float x[4] = {s0[0], s0[1], s1[0], s1[1]};
       const int kx[4] = {2 * tq, 2 * tq + 1, 8 + 2 * tq, 9 + 2 * tq};
-      float bm = -INFINITY;
+      float p[NR][4];
+      bool rescale = false;
+      float alpha[NR];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        x[e] = kx[e] < nk ? x[e] * scale_log2 : -INFINITY;
-        bm = fmaxf(bm, x[e]);
-      }
-      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));  // block max of head gq (key 0 is valid)
-      // lazy rescale: the reference max moves only when the block max exceeds it by more than 8
-      float alpha = 1.f;
-      if (bm > mrow + 8.f || mrow == -INFINITY) {
-        alpha = (mrow == -INFINITY) ? 0.f : fast_exp2(mrow - bm);
-        mrow = bm;
-      }
-      if (__any_sync(0xffffffffu, alpha != 1.f)) {
-        lrow *= alpha;
+      for (int r = 0; r < NR; ++r) {
+        float x[4] = {s0[2 * r], s0[2 * r + 1], s1[2 * r], s1[2 * r + 1]};
+        // visible: inside the chunk and at or before the row's causal limit
+        const int vis = valid[r] ? min(nk, lim[r] - bk * kDecBlk + 1) : 0;
+        float bm = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < D / 8; ++j) {
-          o[j][0] *= alpha;
-          o[j][1] *= alpha;
+        for (int e = 0; e < 4; ++e) {
+          x[e] = kx[e] < vis ? x[e] * scale_log2 : -INFINITY;
+          bm = fmaxf(bm, x[e]);
+        }
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));  // block max of the row
+        // lazy rescale: the reference max moves only when the block max exceeds it by more than 8
+        alpha[r] = 1.f;
+        if (bm > mrow[r] + 8.f || (mrow[r] == -INFINITY && bm != -INFINITY)) {
+          alpha[r] = (mrow[r] == -INFINITY) ? 0.f : fast_exp2(mrow[r] - bm);
+          mrow[r] = bm;
+        }
+        rescale = rescale || alpha[r] != 1.f;
+        const float m_use = mrow[r] == -INFINITY ? 0.f : mrow[r];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) p[r][e] = fast_exp2(x[e] - m_use);  // 2^(-inf) = 0 for hidden keys
+      }
+      if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          lrow[r] *= alpha[r];
+#pragma unroll
+          for (int j = 0; j < D / 8; ++j) {
+            o[j][2 * r] *= alpha[r];
+            o[j][2 * r + 1] *= alpha[r];
+          }
         }
       }
-      float p[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        p[e] = head ? fast_exp2(x[e] - mrow) : 0.f;  // 2^(-inf) = 0 for keys past the block's end
-        lrow += p[e];
-      }
-      const uint32_t pa0 = pack_bf16(p[0], p[1]), pa2 = pack_bf16(p[2], p[3]);
+      for (int r = 0; r < NR; ++r) lrow[r] += (p[r][0] + p[r][1]) + (p[r][2] + p[r][3]);
+      const uint32_t pa0 = pack_bf16(p[0][0], p[0][1]), pa2 = pack_bf16(p[0][2], p[0][3]);
+      const uint32_t pa1 = NR == 2 ? pack_bf16(p[NR - 1][0], p[NR - 1][1]) : 0u;
+      const uint32_t pa3 = NR == 2 ? pack_bf16(p[NR - 1][2], p[NR - 1][3]) : 0u;
       // O += P V over pairs of 8-column tiles
 #pragma unroll
       for (int jp = 0; jp < D / 16; ++jp) {
         uint32_t v0, v1, v2, v3;  // matrices: keys 8 (mi % 2) + ri, head dims 16 jp + 8 (mi / 2) ..
         ldsm_x4_trans(vb + dec_sw<D>(ri + 8 * (mi & 1), 16 * jp + 8 * (mi >> 1)), v0, v1, v2, v3);
-        mma_16816(o[2 * jp], pa0, 0u, pa2, 0u, v0, v1);
-        mma_16816(o[2 * jp + 1], pa0, 0u, pa2, 0u, v2, v3);
+        mma_16816(o[2 * jp], pa0, pa1, pa2, pa3, v0, v1);
+        mma_16816(o[2 * jp + 1], pa0, pa1, pa2, pa3, v2, v3);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty + s);
@@ -441,49 +506,60 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
     gb += it.nblk;
     __syncwarp();
     if (ok && lane == 0) mbar_arrive(q_empty + qbuf);  // done with this item's query rows
-    lrow += __shfl_xor_sync(0xffffffffu, lrow, 1);
-    lrow += __shfl_xor_sync(0xffffffffu, lrow, 2);
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      lrow[r] += __shfl_xor_sync(0xffffffffu, lrow[r], 1);
+      lrow[r] += __shfl_xor_sync(0xffffffffu, lrow[r], 2);
+    }
     // Merge the four warps' triples (a warp that saw no block of the item holds the identity).
     // Named barrier 1: warps 1-3 have deposited; barrier 2: warp 0 has read the deposits, so they
     // may be overwritten. Every compute warp passes both for every item, also after a failed wait.
     if (warp > 0) {
       if (qi > 1) named_barrier(2, 128);
-      if (head) {
-        float* dw = dep + ((warp - 1) * GT + gq) * D;
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        if (!valid[r]) continue;
+        const int row = gq + 8 * r;
+        float* dw = dep + ((warp - 1) * RM + row) * D;
         if (tq == 0) {
-          dep_m[(warp - 1) * 4 + gq] = mrow;
-          dep_l[(warp - 1) * 4 + gq] = lrow;
+          dep_m[(warp - 1) * RM + row] = mrow[r];
+          dep_l[(warp - 1) * RM + row] = lrow[r];
         }
 #pragma unroll
-        for (int j = 0; j < D / 8; ++j) *reinterpret_cast<float2*>(dw + 8 * j + 2 * tq) = make_float2(o[j][0], o[j][1]);
+        for (int j = 0; j < D / 8; ++j)
+          *reinterpret_cast<float2*>(dw + 8 * j + 2 * tq) = make_float2(o[j][2 * r], o[j][2 * r + 1]);
       }
       named_barrier_arrive(1, 128);
     } else {
       named_barrier(1, 128);
-      if (head) {
-        float M = mrow;
 #pragma unroll
-        for (int w = 0; w < 3; ++w) M = fmaxf(M, dep_m[w * 4 + gq]);
+      for (int r = 0; r < NR; ++r) {
+        if (!valid[r]) continue;
+        const int row = gq + 8 * r;
+        float M = mrow[r];
+#pragma unroll
+        for (int w = 0; w < 3; ++w) M = fmaxf(M, dep_m[w * RM + row]);
         float e0 = 0.f, ew[3] = {0.f, 0.f, 0.f};
         if (M != -INFINITY) {
-          e0 = mrow == -INFINITY ? 0.f : fast_exp2(mrow - M);
+          e0 = mrow[r] == -INFINITY ? 0.f : fast_exp2(mrow[r] - M);
 #pragma unroll
           for (int w = 0; w < 3; ++w) {
-            const float mw = dep_m[w * 4 + gq];
+            const float mw = dep_m[w * RM + row];
             ew[w] = mw == -INFINITY ? 0.f : fast_exp2(mw - M);
           }
         }
-        float Lsum = e0 * lrow;
+        float Lsum = e0 * lrow[r];
 #pragma unroll
-        for (int w = 0; w < 3; ++w) Lsum = fmaf(ew[w], dep_l[w * 4 + gq], Lsum);
-        const long long slot = (static_cast<long long>(it.n) * Hq + it.h0 + gq) * max_splits + it.c;
+        for (int w = 0; w < 3; ++w) Lsum = fmaf(ew[w], dep_l[w * RM + row], Lsum);
+        const int tok = it.tq0 + row / dq.GT, h = it.h0 + row % dq.GT;
+        const long long slot = ((static_cast<long long>(it.n) * dq.q_len + tok) * Hq + h) * max_splits + it.c;
         float* dst = part_o + slot * D;
 #pragma unroll
         for (int j = 0; j < D / 8; ++j) {
-          float a0 = e0 * o[j][0], a1 = e0 * o[j][1];
+          float a0 = e0 * o[j][2 * r], a1 = e0 * o[j][2 * r + 1];
 #pragma unroll
           for (int w = 0; w < 3; ++w) {
-            const float2 y = *reinterpret_cast<const float2*>(dep + (w * GT + gq) * D + 8 * j + 2 * tq);
+            const float2 y = *reinterpret_cast<const float2*>(dep + (w * RM + row) * D + 8 * j + 2 * tq);
             a0 = fmaf(ew[w], y.x, a0);
             a1 = fmaf(ew[w], y.y, a1);
           }
@@ -501,23 +577,26 @@ __global__ void __launch_bounds__(kDecThreads, kDecCtasPerSm)
   griddep_launch_dependents();
 }
 
+// Merge of the partial triples of one output row (stream n, query token t, query head h): one warp.
 template <int D>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __restrict__ part_o,
                                                              const float* __restrict__ part_ml,
                                                              const DecKV kv,
                                                              const int* __restrict__ num_splits, int max_splits,
-                                                             int N, int Hq, uint16_t* __restrict__ o,
+                                                             int N, int q_len, int Hq, uint16_t* __restrict__ o,
                                                              float* __restrict__ lse) {
   constexpr int DPL = D / 32;
   griddep_wait();  // the split kernel's partial triples
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long gw = static_cast<long long>(blockIdx.x) * 4 + warp;
-  if (gw >= static_cast<long long>(N) * Hq) return;
-  const int n = static_cast<int>(gw / Hq), h = static_cast<int>(gw % Hq);
+  const long long gw = static_cast<long long>(blockIdx.x) * 4 + warp;  // (n, t, h), h fastest
+  if (gw >= static_cast<long long>(N) * q_len * Hq) return;
+  const int h = static_cast<int>(gw % Hq);
+  const long long nt = gw / Hq;
+  const int n = static_cast<int>(nt / q_len), tok = static_cast<int>(nt % q_len);
   int st0, L;
   dec_stream(kv, n, st0, L);
   const int C = stream_splits(num_splits, n, L, max_splits);
-  const long long slot0 = (static_cast<long long>(n) * Hq + h) * max_splits;
+  const long long slot0 = gw * max_splits;
   // The first 16 partial rows are loaded before anything else, so their loads and those of the
   // (m, l) pairs are in flight together; lane c holds the pair of chunk c and c + 32 (max_splits
   // <= 64).
@@ -582,7 +661,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
       for (int e = 0; e < DPL; ++e) acc[e] = fmaf(wv[u], y4[u][e], acc[e]);
   }
   const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
-  uint16_t* dst = o + (static_cast<long long>(n) * Hq + h) * D + lane * DPL;
+  uint16_t* dst = o + gw * D + lane * DPL;  // o [N, q_len, Hq, D]: row (n, t, h) is row gw
   if constexpr (DPL == 4) {
     uint2 w;
     w.x = pack_bf16(acc[0] * inv, acc[1] * inv);
@@ -591,41 +670,66 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
   } else {
     *reinterpret_cast<uint32_t*>(dst) = pack_bf16(acc[0] * inv, acc[1] * inv);
   }
-  if (lane == 0 && lse) lse[static_cast<long long>(n) * Hq + h] = Lt > 0.f ? (M + log2f(Lt)) * kLn2 : -INFINITY;
+  // lse [N, Hq, q_len]
+  if (lane == 0 && lse)
+    lse[(static_cast<long long>(n) * Hq + h) * q_len + tok] = Lt > 0.f ? (M + log2f(Lt)) * kLn2 : -INFINITY;
 }
 
-template <int D, int GT>
-cudaError_t launch_split(const DecodeProblem& p, const void* q, const void* k, const void* v,
+template <int D, int RM>
+cudaError_t launch_split(const DecodeProblem& p, const DecQ& dq, const void* q, const void* k, const void* v,
                          const CUtensorMap& mk, const CUtensorMap& mv, const DecKV& kv, const int* num_splits,
                          float* part_o, float* part_ml, cudaStream_t st) {
-  using C = DecCfg<D>;
-  const int npass = (p.Hq / p.Hkv) / GT;
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, GT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  using C = DecCfg<D, RM>;
+  const int NG = p.Hkv * ((p.Hq / p.Hkv) / dq.GT) * dq.ntp;
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, RM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  // a persistent grid: kDecCtasPerSm CTAs per SM, capped by the number of item slots
+  // a persistent grid: as many CTAs as fit on the SMs, capped by the number of item slots
   int dev = 0, sms = 0;
   e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  const long long n_slots = static_cast<long long>(p.N) * p.Hkv * npass * p.max_splits;
-  const unsigned grid = static_cast<unsigned>(std::min<long long>(n_slots, static_cast<long long>(sms) * kDecCtasPerSm));
+  const long long n_slots = static_cast<long long>(p.N) * NG * p.max_splits;
+  const unsigned grid = static_cast<unsigned>(
+      std::min<long long>(n_slots, static_cast<long long>(sms) * dec_ctas_per_sm<RM>()));
   {
     LaunchScope ls("decode_split", st);
-    decode_split_kernel<D, GT><<<grid, kDecThreads, C::kSmemBytes, st>>>(
+    decode_split_kernel<D, RM><<<grid, kDecThreads, C::kSmemBytes, st>>>(
         mk, mv, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v),
-        kv, p.N, num_splits, p.max_splits, p.Hq, p.Hkv, p.scale * kLog2e, part_o, part_ml,
+        kv, dq, p.N, num_splits, p.max_splits, p.Hq, p.Hkv, p.scale * kLog2e, part_o, part_ml,
         device_status_ptr());
   }
   return cudaGetLastError();
+}
+
+// Rows of an item: GT query heads (4, 2 or 1, a divisor of the group size) x TQ query tokens. One
+// token per stream keeps to the 4-row variant; more tokens fill up to 16 rows.
+DecQ decode_rows(int G, int q_len, int& rm) {
+  DecQ dq;
+  dq.q_len = q_len;
+  dq.GT = (G % 4 == 0) ? 4 : ((G % 2 == 0) ? 2 : 1);
+  if (q_len * dq.GT <= 4) {
+    rm = 4;
+    dq.TQ = q_len;
+  } else {
+    rm = 16;
+    dq.TQ = std::min(q_len, 16 / dq.GT);
+  }
+  dq.ntp = (q_len + dq.TQ - 1) / dq.TQ;
+#ifdef ATTN_FAULT_INJECT
+  dq.fault_block = fault_block_for(2);
+#else
+  dq.fault_block = -1;
+#endif
+  return dq;
 }
 
 template <int D>
 cudaError_t launch_decode_d(const DecodeProblem& p, const void* q, const void* k, const void* v, const DecKV& kv,
                             long long map_rows, const int* num_splits, void* o, float* lse, void* workspace,
                             cudaStream_t st) {
-  const size_t slots = static_cast<size_t>(p.N) * p.Hq * p.max_splits;
+  const size_t slots = static_cast<size_t>(p.N) * p.q_len * p.Hq * p.max_splits;
   float* part_o = static_cast<float*>(workspace);
   float* part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                             ((slots * D * sizeof(float) + 255) & ~static_cast<size_t>(255)));
@@ -636,21 +740,18 @@ cudaError_t launch_decode_d(const DecodeProblem& p, const void* q, const void* k
   if (!make_map_packed_bf16(&mk, k, map_rows, p.Hkv, D, kDecBlk) ||
       !make_map_packed_bf16(&mv, v, map_rows, p.Hkv, D, kDecBlk))
     return cudaErrorInvalidValue;
-  const int G = p.Hq / p.Hkv;
-  cudaError_t e;
-  if (G % 4 == 0)  // at most four query heads per CTA
-    e = launch_split<D, 4>(p, q, k, v, mk, mv, kv, num_splits, part_o, part_ml, st);
-  else if (G % 2 == 0)
-    e = launch_split<D, 2>(p, q, k, v, mk, mv, kv, num_splits, part_o, part_ml, st);
-  else
-    e = launch_split<D, 1>(p, q, k, v, mk, mv, kv, num_splits, part_o, part_ml, st);
+  int rm = 4;
+  const DecQ dq = decode_rows(p.Hq / p.Hkv, p.q_len, rm);
+  cudaError_t e = rm == 4 ? launch_split<D, 4>(p, dq, q, k, v, mk, mv, kv, num_splits, part_o, part_ml, st)
+                          : launch_split<D, 16>(p, dq, q, k, v, mk, mv, kv, num_splits, part_o, part_ml, st);
   if (e != cudaSuccess) return e;
-  const long long warps = static_cast<long long>(p.N) * p.Hq;
+  const long long warps = static_cast<long long>(p.N) * p.q_len * p.Hq;
   {
     LaunchScope ls("decode_combine", st);
     const cudaError_t e2 =
         launch_dependent(decode_combine_kernel<D>, dim3(static_cast<unsigned>((warps + 3) / 4)), dim3(128), 0, st,
-                         part_o, part_ml, kv, num_splits, p.max_splits, p.N, p.Hq, static_cast<uint16_t*>(o), lse);
+                         part_o, part_ml, kv, num_splits, p.max_splits, p.N, p.q_len, p.Hq,
+                         static_cast<uint16_t*>(o), lse);
     if (e2 != cudaSuccess) return e2;
   }
   return cudaGetLastError();

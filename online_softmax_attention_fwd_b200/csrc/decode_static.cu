@@ -10,8 +10,10 @@
 //
 // Rules of use, all stated in include/attn.h:
 //  * Every GPU that loads the library holds the 16 MiB array until the process exits.
-//  * The first call on a device looks up the array's device address (cudaGetSymbolAddress, once
-//    per device, with that device current); make that first call before any stream capture.
+//  * The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
+//    that device current) and keeps it for the device's current context; the first call after that
+//    context has been torn down and created again (cudaDeviceReset) looks it up again, since the
+//    module may then be loaded elsewhere. Make each such first call before any stream capture.
 //  * Problems whose partial triples need more than 16 MiB are rejected with ATTN_ERR_WORKSPACE
 //    before anything is launched.
 //  * All calls share the one array, and each call leaves its partial triples there. Nothing needs
@@ -29,33 +31,30 @@ namespace attn {
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(16) << 20;  // 16 MiB per device
-constexpr int kMaxStaticDevices = 64;
 
 // The scratch itself. Host code must never pass this name to a kernel: on the host it is only a
 // stand-in, not a device address. The device address is looked up below.
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
 
 std::mutex g_static_mu;
-void* g_static_ptr[kMaxStaticDevices];  // device address of g_decode_scratch, per device
+ContextCache g_static_cache;  // device address of g_decode_scratch, per device and context
 
-// Once per device, with that device current: the device address of the scratch array.
+// The device address of the scratch array on the current device: looked up once per device and
+// context, with that device current.
 cudaError_t static_scratch_ptr(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxStaticDevices) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= kMaxCachedDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lk(g_static_mu);
-  if (!g_static_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess) return e;
-    g_static_ptr[dev] = p;
-  }
-  *out = g_static_ptr[dev];
+  if (g_static_cache.lookup(dev, out)) return cudaSuccess;
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_decode_scratch);
+  if (e != cudaSuccess) return e;
+  g_static_cache.store(dev, p);
+  *out = p;
   return cudaSuccess;
 }
-
-bool aligned16_static(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
 }  // namespace attn
@@ -65,25 +64,17 @@ extern "C" attn_status_t attn_decode_splitkv_static(const void* q, const void* k
                                                     int max_splits, void* o, float* lse, int N, int Hq,
                                                     int Hkv, int D, float scale, attn_stream_t stream) {
   using namespace attn;
-  if (N <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
-  if (max_splits < 1 || max_splits > 64) return ATTN_ERR_INVALID_ARG;
-  if (N > 65535 || static_cast<long long>(N) * Hq >= (1ll << 31)) return ATTN_ERR_INVALID_ARG;
-  if (!q || !k || !v || !kv_offsets || !o) return ATTN_ERR_INVALID_ARG;
-  if (!aligned16_static(q) || !aligned16_static(k) || !aligned16_static(v) || !aligned16_static(kv_offsets) ||
-      !aligned16_static(o) || (num_splits && !aligned16_static(num_splits)) || (lse && !aligned16_static(lse)))
-    return ATTN_ERR_ALIGNMENT;
-  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  // the same argument checks as attn_decode_splitkv; only the scratch differs
+  attn_status_t s = check_decode_args(q, k, v, kv_offsets, num_splits, max_splits, o, lse, N, Hq, Hkv, D);
+  if (s != ATTN_OK) return s;
   if (decode_workspace_bytes(N, Hq, D, max_splits) > kStaticScratchBytes) return ATTN_ERR_WORKSPACE;
-  int dev = -1, major = 0, minor = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-      major * 10 + minor != 100)
-    return ATTN_ERR_UNSUPPORTED;
+  if (!device_is_sm100()) return ATTN_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   if (static_scratch_ptr(&scratch) != cudaSuccess) return ATTN_ERR_LAUNCH;
-  const DecodeProblem p{N, Hq, Hkv, D, max_splits, scale};
+  const DecodeProblem p{N, Hq, Hkv, D, max_splits, scale, 1};
   const cudaError_t e =
       launch_decode(p, q, k, v, kv_offsets, num_splits, o, lse, scratch, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+  if (e != cudaSuccess) return ATTN_ERR_LAUNCH;
+  set_last_path(2, "decode_splitkv_static_mma16816");
+  return ATTN_OK;
 }

@@ -56,10 +56,14 @@ constexpr int kBN = 128;   // keys per block
 constexpr int kThreads = 320;
 constexpr int kAtom = 128 * 128;  // 128 rows x 128 bytes (16 KB)
 
-template <int D>
+// F8: e4m3 Q, K, V (one byte per element, D = 128 only) instead of bf16.
+template <int D, bool F8 = false>
 struct FwdCfg {
-  static constexpr int kAtoms = D / 64;              // 64-element column atoms per row
+  static constexpr int kElt = F8 ? 1 : 2;             // bytes per element
+  static constexpr int kAtomElts = 128 / kElt;        // elements per 128-byte swizzle row
+  static constexpr int kAtoms = D / kAtomElts;        // column atoms per row
   static constexpr int kTileBytes = kAtoms * kAtom;  // one 128 x D tile (Q, K or V)
+  static constexpr int kKStep = 32 / kElt;            // K elements per MMA instruction (32 bytes)
   static constexpr int kKStages = (D == 128) ? 2 : 4;
   static constexpr int kVStages = (D == 128) ? 2 : 4;
   static constexpr int kOffQ = 0;                                      // [2 tiles]
@@ -75,9 +79,10 @@ struct FwdCfg {
 };
 
 struct FwdArgs {
-  int B, Hq, Hkv, Sq, Sk;
+  int B, Hq, Hkv, Sq, Sk;  // packed batches: Sq, Sk are the longest sequence's lengths
   int causal;
-  float scale_log2;  // softmax scale * log2(e)
+  float scale_log2;  // softmax scale * log2(e) (FP8: times the Q and K scales)
+  float o_scale;     // O multiplier at the end (FP8: the V scale; 1 for bf16)
   // A work item is two 128-row query tiles that read the same K/V blocks. With head_pairs, the two
   // tiles are the same rows of query heads 2 hs and 2 hs + 1 (one key/value group, as the head
   // count ratio is even); otherwise they are rows 256 s .. 256 s + 255 of one head.
@@ -87,7 +92,33 @@ struct FwdArgs {
   uint16_t* o;
   float* lse;
   int* status;
+  // Packed batches of sequences of different lengths: sequence b owns query rows cu_q[b] ..
+  // cu_q[b + 1] - 1 of q / o ([Tq, Hq, D]) and key rows cu_k[b] .. cu_k[b + 1] - 1 of k / v, and lse
+  // is [Hq, Tq]. Null for the dense [B, S, H, D] layout.
+  const int* cu_q;
+  const int* cu_k;
+  int Tq, Tk;
+  int fault_block;  // test-only fault-injection build: CTA 0 skips this K load (-1: none)
 };
+
+// Lengths and first packed rows of sequence b (dense: every sequence has Sq / Sk rows). Offsets
+// are device data, so they are checked where they are used: a sequence whose rows fall outside the
+// packed tensors, or that is longer than the bound the host passed, is not touched (it counts as
+// empty) and the device status records ATTN_ERR_INVALID_ARG.
+struct SeqSpan {
+  int Sq, Sk, q0, k0;
+};
+__device__ __forceinline__ SeqSpan seq_span(const FwdArgs& a, int b) {
+  if (a.cu_q) {
+    const int q0 = a.cu_q[b], q1 = a.cu_q[b + 1], k0 = a.cu_k[b], k1 = a.cu_k[b + 1];
+    if (q0 < 0 || q1 < q0 || q1 > a.Tq || q1 - q0 > a.Sq || k0 < 0 || k1 < k0 || k1 > a.Tk || k1 - k0 > a.Sk) {
+      record_status(a.status, kStatusBadArg);
+      return SeqSpan{0, 0, 0, 0};
+    }
+    return SeqSpan{q1 - q0, k1 - k0, q0, k0};
+  }
+  return SeqSpan{a.Sq, a.Sk, b * a.Sq, b * a.Sk};
+}
 
 __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
   // Bounded wait that ignores the abort flag: used only to let this thread's own in-flight async
@@ -99,10 +130,10 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
 }
 
 // Number of 128-key blocks some row of the 128-row tile starting at `qs` can see.
-__device__ __forceinline__ int tile_blocks(const FwdArgs& a, int qs) {
-  if (qs >= a.Sq) return 0;
-  int kv_end = a.Sk;
-  if (a.causal) kv_end = min(a.Sk, qs + kBM + a.Sk - a.Sq);
+__device__ __forceinline__ int tile_blocks(const SeqSpan& sp, int causal, int qs) {
+  if (qs >= sp.Sq) return 0;
+  int kv_end = sp.Sk;
+  if (causal) kv_end = min(sp.Sk, qs + kBM + sp.Sk - sp.Sq);
   return kv_end > 0 ? (kv_end + kBN - 1) / kBN : 0;
 }
 
@@ -113,11 +144,14 @@ __device__ __forceinline__ int fwd_item_index(int k, int c, int G, int n_items) 
   return i < n_items ? i : -1;
 }
 
-template <int D>
+// One CTA per SM. Its 10 warps are dealt to the SM's four sub-partitions (three on some), and each
+// sub-partition has 16 K registers: at most 168 registers per thread, which the compiler derives
+// from these bounds.
+template <int D, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + C::kOffQ;
@@ -145,14 +179,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   // item i: row position n_slots - 1 - i / BH (the longest items first under a causal mask) of head
   // set i % BH; tile t covers head h + t dh, rows q0 + t dq
   const int dh = a.head_pairs ? 1 : 0, dq = a.head_pairs ? 0 : kBM;
-  auto item_of = [&](int i, int& b, int& h, int& q0, int& n0, int& n1) {
+  // TMA coordinates: dense tensors are 4-D maps (D, H, S, B); packed ones are (D, H, T, 1), where a
+  // sequence's rows start at its first packed row (boxes may run into the next sequence's rows:
+  // those keys are masked, their values weighted 0, and those query rows are not stored)
+  auto item_of = [&](int i, int& b, int& h, int& q0, int& n0, int& n1, SeqSpan& sp) {
     const int bh = i % BH, slot = a.n_slots - 1 - i / BH;
     b = bh / a.n_hsets;
     h = (bh % a.n_hsets) * (a.head_pairs ? 2 : 1);
     q0 = slot * (a.head_pairs ? kBM : 2 * kBM);
-    n0 = tile_blocks(a, q0);
-    n1 = tile_blocks(a, q0 + dq);
+    sp = seq_span(a, b);
+    n0 = tile_blocks(sp, a.causal, q0);
+    n1 = tile_blocks(sp, a.causal, q0 + dq);
   };
+  const bool packed = a.cu_q != nullptr;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -193,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 8) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      constexpr uint32_t kTx = kBM * D * 2;
+      constexpr uint32_t kTx = kBM * D * C::kElt;
       long long kvb = 0;  // K/V blocks issued so far (ring position)
       int qk = 0;         // items with any block so far
       bool ok = true;
@@ -201,10 +240,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int i = fwd_item_index(k, cta, G, n_items);
         if (i < 0) break;
         int b, h, q0, n0, n1;
-        item_of(i, b, h, q0, n0, n1);
+        SeqSpan sp;
+        item_of(i, b, h, q0, n0, n1, sp);
         const int nmax = max(n0, n1);
         if (nmax == 0) continue;
         const int g = h / (a.Hq / a.Hkv);
+        const int qrow0 = packed ? sp.q0 : 0, krow0 = packed ? sp.k0 : 0, bc = packed ? 0 : b;
         // this item's Q tiles once the previous item's last S has read the buffer
         if (!mbar_wait(q_empty, (qk & 1) ^ 1, abort, a.status)) break;
         mbar_arrive_expect_tx(q_full, (n0 > 0 ? kTx : 0u) + (n1 > 0 ? kTx : 0u));
@@ -213,7 +254,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if ((t == 0 ? n0 : n1) == 0) continue;
 #pragma unroll
           for (int at = 0; at < C::kAtoms; ++at)
-            tma_load_4d(sQ + t * C::kTileBytes + at * kAtom, &tmQ, q_full, at * 64, h + t * dh, q0 + t * dq, b);
+            tma_load_4d(sQ + t * C::kTileBytes + at * kAtom, &tmQ, q_full, at * C::kAtomElts, h + t * dh,
+                        qrow0 + q0 + t * dq, bc);
         }
         ++qk;
         for (int j = 0; j < nmax; ++j) {
@@ -223,10 +265,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(k_full + sk, kTx);
+#ifdef ATTN_FAULT_INJECT
+          const bool skip = cta == 0 && gj == a.fault_block;  // the MMA warp's wait for it runs out
+#else
+          constexpr bool skip = false;
+#endif
+          if (!skip) {
+            mbar_arrive_expect_tx(k_full + sk, kTx);
 #pragma unroll
-          for (int at = 0; at < C::kAtoms; ++at)
-            tma_load_4d(sK + sk * C::kTileBytes + at * kAtom, &tmK, k_full + sk, at * 64, g, j * kBN, b);
+            for (int at = 0; at < C::kAtoms; ++at)
+              tma_load_4d(sK + sk * C::kTileBytes + at * kAtom, &tmK, k_full + sk, at * C::kAtomElts, g,
+                          krow0 + j * kBN, bc);
+          }
           if (!mbar_wait(v_empty + sv, static_cast<uint32_t>((gj / C::kVStages) & 1) ^ 1, abort, a.status)) {
             ok = false;
             break;
@@ -234,7 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(v_full + sv, kTx);
 #pragma unroll
           for (int at = 0; at < C::kAtoms; ++at)
-            tma_load_4d(sV + sv * C::kTileBytes + at * kAtom, &tmV, v_full + sv, at * 64, g, j * kBN, b);
+            tma_load_4d(sV + sv * C::kTileBytes + at * kAtom, &tmV, v_full + sv, at * C::kAtomElts, g,
+                        krow0 + j * kBN, bc);
         }
         kvb += nmax;
       }
@@ -249,8 +300,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
     // the whole warp runs the loop; one elected lane issues each MMA
-    constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, 0, 0);
-    constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, D, 0, 1);
+    constexpr uint32_t kIdescS = F8 ? idesc_e4m3_f32(kBM, kBN, 0, 0) : idesc_bf16_f32(kBM, kBN, 0, 0);
+    constexpr uint32_t kIdescO = F8 ? idesc_e4m3_f32(kBM, D, 0, 1) : idesc_bf16_f32(kBM, D, 0, 1);
     // base descriptors, built once; each MMA only moves the start address
     const uint64_t dQ0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
     const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);
@@ -281,9 +332,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dK = sdesc_advance(dK0, static_cast<uint32_t>(gj % C::kKStages) * C::kTileBytes);
       const uint64_t dQ = sdesc_advance(dQ0, t * C::kTileBytes);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
-        umma_ss_warp(tmem + C::colS(t), sdesc_advance(dQ, off), sdesc_advance(dK, off), kIdescS, kk > 0);
+      for (int kk = 0; kk < D / C::kKStep; ++kk) {
+        const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;  // 32 bytes of K per instruction
+        if constexpr (F8)
+          umma_ss_warp_f8(tmem + C::colS(t), sdesc_advance(dQ, off), sdesc_advance(dK, off), kIdescS, kk > 0);
+        else
+          umma_ss_warp(tmem + C::colS(t), sdesc_advance(dQ, off), sdesc_advance(dK, off), kIdescS, kk > 0);
       }
       umma_commit_warp(s_full + t);
     };
@@ -291,7 +345,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i = fwd_item_index(k, cta, G, n_items);
       if (i < 0) break;
       int b, h, q0, n0, n1;
-      item_of(i, b, h, q0, n0, n1);
+      SeqSpan sp;
+      item_of(i, b, h, q0, n0, n1, sp);
       const int nmax = max(n0, n1);
       if (nmax == 0) continue;
       const int nt[2] = {n0, n1};
@@ -314,8 +369,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             const uint64_t dV = sdesc_advance(dV0, static_cast<uint32_t>(gj % C::kVStages) * C::kTileBytes);
-            // P (bf16) is the A operand in TMEM, 16 keys = 8 columns per step; each half of the
-            // block's keys goes as soon as the softmax has written its P
+            // P is the A operand in TMEM, 8 columns per instruction (16 bf16 keys, or 32 e4m3 keys);
+            // each half of the block's keys goes as soon as the softmax has written its P
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
               if ((hf == 0 && !wait_v(gj)) ||
@@ -324,10 +379,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
               }
               tc_fence_after();
+              constexpr int kPerHalf = 64 / C::kKStep;  // instructions per 64 keys
 #pragma unroll
-              for (int kk = 4 * hf; kk < 4 * hf + 4; ++kk)
-                umma_ts_warp(tmem + C::colO(t), tmem + C::colS(t) + kk * 8, sdesc_advance(dV, kk * 16 * 128),
-                             kIdescO, (j > 0 || kk > 0));
+              for (int kk = kPerHalf * hf; kk < kPerHalf * hf + kPerHalf; ++kk) {
+                if constexpr (F8)
+                  umma_ts_warp_f8(tmem + C::colO(t), tmem + C::colS(t) + kk * 8,
+                                  sdesc_advance(dV, kk * C::kKStep * 128), kIdescO, (j > 0 || kk > 0));
+                else
+                  umma_ts_warp(tmem + C::colO(t), tmem + C::colS(t) + kk * 8, sdesc_advance(dV, kk * C::kKStep * 128),
+                               kIdescO, (j > 0 || kk > 0));
+              }
             }
             if (!ok) break;
             if (j == nt[t] - 1) umma_commit_warp(o_done + t);
@@ -377,12 +438,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i = fwd_item_index(k, cta, G, n_items);
       if (i < 0) break;
       int b, h, q0, n0, n1;
-      item_of(i, b, h, q0, n0, n1);
+      SeqSpan sp;
+      item_of(i, b, h, q0, n0, n1, sp);
       const int n_kv = t == 0 ? n0 : n1;
       h += t * dh;
       const int qrow = q0 + t * dq + row;
-      int row_limit = a.Sk - 1;  // largest visible key index for this row
-      if (a.causal) row_limit = min(row_limit, qrow + a.Sk - a.Sq);
+      int row_limit = sp.Sk - 1;  // largest visible key index for this row
+      if (a.causal) row_limit = min(row_limit, qrow + sp.Sk - sp.Sq);
       float m = -INFINITY, l = 0.f;
       for (int j = 0; ok && j < n_kv; ++j) {
         if (!wait_warp(s_full + t, static_cast<uint32_t>((sb + j) & 1))) {
@@ -420,12 +482,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float m_use = (m == -INFINITY) ? 0.f : m;
         // P = 2^(scale s - m) as bf16 pairs over the first 64 columns of S: keys 0-63 first (P columns
-        // 0-31), released to the P V MMA at once, then keys 64-127 (ex2 of a masked -inf is 0)
+        // 0-31), released to the P V MMA at once, then keys 64-127 (ex2 of a masked -inf is 0). FP8:
+        // e4m3 quadruples over the first 32 columns (keys 0-63 in columns 0-15). With the lazy
+        // rescale P <= 2^8, inside e4m3's range (448).
         const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), nm2 = f2_pack(-m_use, -m_use);
         uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};  // four packed sum chains
   #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           uint32_t pk[32];
+          float pprev = 0.f, pprev1 = 0.f;
   #pragma unroll
           for (int c = 64 * hf; c < 64 * hf + 64; c += 2) {
             float x0, x1, p0, p1;
@@ -433,10 +498,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             p0 = fast_exp2(x0);
             p1 = fast_exp2(x1);
             rs2[(c >> 1) & 3] = f2_add(rs2[(c >> 1) & 3], f2_pack(p0, p1));
-            pk[(c - 64 * hf) / 2] = pack_bf16(p0, p1);
+            if constexpr (F8) {
+              if (c & 2) pk[(c - 64 * hf) / 4] = pack_e4m3x4(pprev, pprev1, p0, p1);
+              pprev = p0;
+              pprev1 = p1;
+            } else {
+              pk[(c - 64 * hf) / 2] = pack_bf16(p0, p1);
+            }
           }
-          tmem_st16(tS + 32 * hf, pk);
-          tmem_st16(tS + 32 * hf + 16, pk + 16);
+          if constexpr (F8) {
+            tmem_st16(tS + 16 * hf, pk);
+          } else {
+            tmem_st16(tS + 32 * hf, pk);
+            tmem_st16(tS + 32 * hf + 16, pk + 16);
+          }
           // S of block j is complete, hence so is P V of block j - 1: O may be rescaled now, before
           // the first P V of block j is released.
           if (hf == 0 && j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
@@ -466,9 +541,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool have = ok && n_kv > 0;
       if (have) ok = wait_warp(o_done + t, ct & 1);
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const bool store = qrow < a.Sq;
-      uint16_t* orow = a.o + ((static_cast<long long>(b) * a.Sq + qrow) * a.Hq + h) * D;
+      const float inv = l > 0.f ? a.o_scale / l : 0.f;
+      const bool store = qrow < sp.Sq;
+      uint16_t* orow = a.o + ((static_cast<long long>(sp.q0) + qrow) * a.Hq + h) * D;
       uint32_t orr[D];
       if (have && ok) {
 #pragma unroll
@@ -499,8 +574,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(orow + c0) = w0;
           *reinterpret_cast<uint4*>(orow + c0 + 8) = w1;
         }
-        a.lse[(static_cast<long long>(b) * a.Hq + h) * a.Sq + qrow] =
-            l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+        const long long li = packed ? static_cast<long long>(h) * a.Tq + sp.q0 + qrow
+                                    : (static_cast<long long>(b) * a.Hq + h) * a.Sq + qrow;
+        a.lse[li] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
       }
     }
   }
@@ -516,15 +592,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------------------------
 // host side: tensor maps and launch
 // ---------------------------------------------------------------------------------------------
-template <int D>
+template <int D, bool F8>
 cudaError_t launch_fwd_sm100_d(const Problem& p, const void* q, const void* k, const void* v, void* o, float* lse,
                                cudaStream_t st) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, F8>;
   CUtensorMap mq, mk, mv;
-  if (!make_map_bf16_sw128(&mq, q, p.B, p.Sq, p.Hq, D, kBM) ||
-      !make_map_bf16_sw128(&mk, k, p.B, p.Sk, p.Hkv, D, kBN) || !make_map_bf16_sw128(&mv, v, p.B, p.Sk, p.Hkv, D, kBN))
+  const bool packed = p.cu_q != nullptr;
+  // packed batches: one sequence of Tq (Tk) rows as far as the maps are concerned
+  const int mB = packed ? 1 : p.B, mSq = packed ? p.Tq : p.Sq, mSk = packed ? p.Tk : p.Sk;
+  auto make = [&](CUtensorMap* m, const void* base, int S, int H, int rows) {
+    return F8 ? make_map_u8_sw128(m, base, mB, S, H, D, rows) : make_map_bf16_sw128(m, base, mB, S, H, D, rows);
+  };
+  if (!make(&mq, q, mSq, p.Hq, kBM) || !make(&mk, k, mSk, p.Hkv, kBN) || !make(&mv, v, mSk, p.Hkv, kBN))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  cudaError_t e =
+      cudaFuncSetAttribute(fwd_sm100_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   FwdArgs a;
   a.B = p.B;
@@ -533,13 +615,23 @@ cudaError_t launch_fwd_sm100_d(const Problem& p, const void* q, const void* k, c
   a.Sq = p.Sq;
   a.Sk = p.Sk;
   a.causal = p.causal;
-  a.scale_log2 = p.scale * kLog2e;
+  a.scale_log2 = p.scale * p.qk_scale * kLog2e;
+  a.o_scale = p.v_scale;
   a.head_pairs = (p.Hq / p.Hkv) % 2 == 0 ? 1 : 0;
   a.n_slots = a.head_pairs ? (p.Sq + kBM - 1) / kBM : (p.Sq + 2 * kBM - 1) / (2 * kBM);
   a.n_hsets = a.head_pairs ? p.Hq / 2 : p.Hq;
   a.o = static_cast<uint16_t*>(o);
   a.lse = lse;
   a.status = device_status_ptr();
+  a.cu_q = p.cu_q;
+  a.cu_k = p.cu_k;
+  a.Tq = p.Tq;
+  a.Tk = p.Tk;
+#ifdef ATTN_FAULT_INJECT
+  a.fault_block = fault_block_for(0);
+#else
+  a.fault_block = -1;
+#endif
   // a persistent grid: one CTA per SM, each walking its share of the (head, tile pair) items
   int dev = 0, sms = 0;
   e = cudaGetDevice(&dev);
@@ -549,8 +641,8 @@ cudaError_t launch_fwd_sm100_d(const Problem& p, const void* q, const void* k, c
   const long long n_items = static_cast<long long>(a.n_hsets) * p.B * a.n_slots;
   dim3 grid(static_cast<unsigned>(std::min<long long>(n_items, sms)));
   {
-    LaunchScope ls("fwd_sm100", st);
-    fwd_sm100_kernel<D><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);
+    LaunchScope ls(F8 ? "fwd_sm100_fp8" : "fwd_sm100", st);
+    fwd_sm100_kernel<D, F8><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);
   }
   return cudaGetLastError();
 }
@@ -559,8 +651,14 @@ cudaError_t launch_fwd_sm100_d(const Problem& p, const void* q, const void* k, c
 
 cudaError_t launch_fwd_sm100(const Problem& p, const void* q, const void* k, const void* v, void* o, float* lse,
                              cudaStream_t st) {
-  if (p.D == 128) return launch_fwd_sm100_d<128>(p, q, k, v, o, lse, st);
-  return launch_fwd_sm100_d<64>(p, q, k, v, o, lse, st);
+  if (p.D == 128) return launch_fwd_sm100_d<128, false>(p, q, k, v, o, lse, st);
+  return launch_fwd_sm100_d<64, false>(p, q, k, v, o, lse, st);
+}
+
+cudaError_t launch_fwd_sm100_fp8(const Problem& p, const void* q, const void* k, const void* v, void* o, float* lse,
+                                 cudaStream_t st) {
+  if (p.D != 128) return cudaErrorInvalidValue;
+  return launch_fwd_sm100_d<128, true>(p, q, k, v, o, lse, st);
 }
 
 }  // namespace attn

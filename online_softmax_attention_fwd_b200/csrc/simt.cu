@@ -1,8 +1,7 @@
 // simt.cu -- CUDA-core (FFMA) attention forward and backward.
 //
 // The fp32 entry points (attn_fwd_f32 / attn_bwd_f32) run these kernels: genuine fp32 arithmetic,
-// no TF32, so that results stay within 1e-5 of the fp64 definition. They are templated on the
-// storage type so the same code also serves as the checked CUDA-core form of the bf16 path.
+// no TF32, so that results stay within 1e-5 of the fp64 definition.
 //
 // Forward: one warp per query row. The keys are visited in chunks of 32 (one key per lane for the
 // score), and the row's state is the online-softmax triple (m, l, o): running max, running sum of
@@ -27,20 +26,11 @@ template <>
 __device__ __forceinline__ float ldf<float>(const float* p) {
   return __ldg(p);
 }
-template <>
-__device__ __forceinline__ float ldf<uint16_t>(const uint16_t* p) {
-  return __uint_as_float(static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short*>(p))) << 16);
-}
 template <typename T>
 __device__ __forceinline__ void stf(T* p, float x);
 template <>
 __device__ __forceinline__ void stf<float>(float* p, float x) {
   *p = x;
-}
-template <>
-__device__ __forceinline__ void stf<uint16_t>(uint16_t* p, float x) {
-  __nv_bfloat16 b = __float2bfloat16_rn(x);
-  *p = *reinterpret_cast<uint16_t*>(&b);
 }
 
 constexpr int kWarps = 4;
@@ -347,19 +337,10 @@ cudaError_t launch_fwd_simt_f32(const Problem& p, const float* q, const float* k
                                 float* lse, cudaStream_t st) {
   return fwd_simt_any<float>(p, q, k, v, o, lse, st);
 }
-cudaError_t launch_fwd_simt_bf16(const Problem& p, const void* q, const void* k, const void* v, void* o,
-                                 float* lse, cudaStream_t st) {
-  return fwd_simt_any<uint16_t>(p, q, k, v, o, lse, st);
-}
 cudaError_t launch_bwd_simt_f32(const Problem& p, const float* q, const float* k, const float* v, const float* o,
                                 const float* lse, const float* dout, float* dq, float* dk, float* dv,
                                 float* delta, cudaStream_t st) {
   return bwd_simt_any<float>(p, q, k, v, o, lse, dout, dq, dk, dv, delta, st);
-}
-cudaError_t launch_bwd_simt_bf16(const Problem& p, const void* q, const void* k, const void* v, const void* o,
-                                 const float* lse, const void* dout, void* dq, void* dk, void* dv, float* delta,
-                                 cudaStream_t st) {
-  return bwd_simt_any<uint16_t>(p, q, k, v, o, lse, dout, dq, dk, dv, delta, st);
 }
 
 }  // namespace attn

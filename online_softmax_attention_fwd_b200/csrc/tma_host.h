@@ -68,4 +68,9 @@ inline bool make_map_bf16_sw128(CUtensorMap* map, const void* base, int B, int S
                        CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// 8-bit [B, S, H, D] (e4m3 codes) with 128-byte swizzle, boxes of 128 head-dim elements x `rows`.
+inline bool make_map_u8_sw128(CUtensorMap* map, const void* base, int B, int S, int H, int D, int rows) {
+  return make_map_bshd(map, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, S, H, D, 128, rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 }  // namespace attn

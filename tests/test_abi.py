@@ -122,3 +122,13 @@ def test_launch_counter_and_last_path_without_gpu(L):
     assert attn.launch_count() >= 0
     assert isinstance(attn.last_path(0), str)
     assert attn.last_path(7) == "none"
+
+
+def test_fault_injection_switch_only_in_the_test_build(L):
+    # libattn.so never exports the test-only switch; the fault-injection build does
+    import subprocess
+    shipped = subprocess.run(["nm", "-D", "--defined-only", build_mod.LIB_PATH], capture_output=True, text=True).stdout
+    test_build = subprocess.run(["nm", "-D", "--defined-only", build_mod.FAULT_LIB_PATH], capture_output=True,
+                                text=True).stdout
+    assert "attn_fault_inject" not in shipped
+    assert "attn_fault_inject" in test_build

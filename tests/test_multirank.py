@@ -55,3 +55,31 @@ def test_single_process_needs_no_process_group():
     import bench
     assert bench.reduce_max(3.0) == 3.0
     assert bench.whole_job_rate(10.0, 4, 1, 2.0) == pytest.approx(20.0)
+
+
+def test_launcher_starts_n_ranks_and_passes_rank0_line():
+    # bench.launch_ranks is what `python bench.py --gpus N` runs when no process group exists; here
+    # it starts two CPU ranks of a stand-in script, which print one line from rank 0 only.
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    probe = os.path.join(root, "tests", "rank_probe.py")
+    code = ("import sys; sys.path.insert(0, %r); import bench; "
+            "sys.exit(bench.launch_ranks(2, %r, ['--steps', '3']))") % (root, probe)
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    out = json.loads(lines[0])
+    assert out["n_gpus"] == 2 and out["max_seconds"] == 2.0 and out["argv"] == ["--steps", "3"]
+
+
+def test_gpus_must_match_an_existing_process_group():
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, WORLD_SIZE="3", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=120, env=env)
+    assert r.returncode == 2 and "does not match" in r.stderr

@@ -13,9 +13,7 @@
 //   bwd_sm100       one CTA per (128-key tile, kv head): loops over the group's query heads x
 //                   64-row query tiles, keeps dK and dV for its keys in TMEM, and adds each tile's
 //                   dQ into the fp32 accumulator;
-//   bwd_dq_convert  dQ = scale * accumulator, rounded to bf16;
-//   bwd_dkv_convert dK, dV of the key tiles that were split over two CTAs (see BwdArgs::n_split),
-//                   from their fp32 sums (only launched when some key tile was split).
+//   bwd_dq_convert  dQ = scale * accumulator, rounded to bf16.
 //
 // The main kernel works on transposed score tiles so that keys sit on the TMEM lanes:
 //   S^T = K Q^T and dP^T = V dO^T            (M = 128 keys, N = 64 query rows, K = D).
@@ -104,11 +102,6 @@ struct BwdArgs {
   const int* cu_k;
   int Tq, Tk;
   int fault_block;  // test-only fault-injection build: CTA (0, 0) skips this Q / dO tile (-1: none)
-  // Load balance: the first n_split key tiles (the heaviest under a causal mask) are each split
-  // over two CTAs by their (query head, query tile) range; both add their partial dK and dV in
-  // fp32 into dkv_acc [B, Hkv, n_split, 2 (dV, dK), 128, D], which bwd_dkv_convert rounds to bf16.
-  int n_split;
-  float* dkv_acc;
 };
 
 // Rows first .. first + len - 1 of sequence b in a packed tensor of T rows: false (and an empty
@@ -131,8 +124,9 @@ __device__ __forceinline__ bool packed_rows(const int* cu, int b, int T, int max
 struct BwdSpan {
   int Sq, Sk, q0, k0;
 };
+template <bool PACKED>
 __device__ __forceinline__ BwdSpan bwd_span(const BwdArgs& a, int b) {
-  if (a.cu_q) {
+  if constexpr (PACKED) {
     BwdSpan s;
     const bool okq = packed_rows(a.cu_q, b, a.Tq, a.Sq, s.q0, s.Sq);
     const bool okk = packed_rows(a.cu_k, b, a.Tk, a.Sk, s.k0, s.Sk);
@@ -141,8 +135,9 @@ __device__ __forceinline__ BwdSpan bwd_span(const BwdArgs& a, int b) {
       return BwdSpan{0, 0, 0, 0};
     }
     return s;
+  } else {
+    return BwdSpan{a.Sq, a.Sk, b * a.Sq, b * a.Sk};
   }
-  return BwdSpan{a.Sq, a.Sk, b * a.Sq, b * a.Sk};
 }
 
 __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
@@ -161,7 +156,7 @@ __device__ __forceinline__ void red_add_v4_f32(float* p, const uint32_t* x) {
 
 // One CTA per SM. Its 14 warps put four on each of the SM's sub-partitions, and each sub-partition
 // has 16 K registers: at most 128 registers per thread, which the compiler derives from these bounds.
-template <int D>
+template <int D, bool PACKED>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -192,17 +187,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = static_cast<int>(blockIdx.x) % a.Hkv;
   const int b = static_cast<int>(blockIdx.x) / a.Hkv;
-  // blockIdx.y -> (key tile, part): the first 2 n_split rows are the two halves of the first n_split
-  // key tiles, then one row per remaining key tile; small key tiles carry the most work under a
-  // causal mask, so the grid is in decreasing order of work
-  const int y = static_cast<int>(blockIdx.y);
-  const bool split = y < 2 * a.n_split;
-  const int kt = split ? (y >> 1) : y - a.n_split;
-  const int part = split ? (y & 1) : 0;
+  const int kt = blockIdx.y;  // key tile; small indices carry the most work under a causal mask
   const int k0 = kt * kBN;
   const int G = a.Hq / a.Hkv;
-  const BwdSpan sp = bwd_span(a, b);
-  const bool packed = a.cu_q != nullptr;
+  const BwdSpan sp = bwd_span<PACKED>(a, b);
+  constexpr bool packed = PACKED;
   // TMA coordinates: dense maps are (D, H, S, B); packed ones (D, H, T, 1) with the sequence's rows
   // starting at its first packed row (rows past its end belong to the next sequence: their lse2 is
   // +inf in the padded per-sequence rows, so their P and dS are 0)
@@ -214,11 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     qt0 = qmin <= 0 ? 0 : qmin / kBM;
   }
   const int n_q = (k0 < sp.Sk && qt0 < n_qt_all) ? n_qt_all - qt0 : 0;
-  // tiles: query head (slow) x query tile (fast), numbered jj = j0 + j over the whole key tile; a
-  // split key tile's first part takes the first ceil(half), the second part the rest
-  const int n_all = G * n_q;
-  const int j0 = part == 0 ? 0 : (n_all + 1) / 2;
-  const int n_it = split ? (part == 0 ? (n_all + 1) / 2 : n_all / 2) : n_all;
+  const int n_it = G * n_q;  // tiles: query head (slow) x query tile (fast)
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -267,8 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued = 0;
       for (int j = 0; j < n_it; ++j) {
         const int s = j % C::kStages;
-        const int h = g * G + (j0 + j) / n_q;
-        const int qt = qt0 + (j0 + j) % n_q;
+        const int h = g * G + j / n_q;
+        const int qt = qt0 + j % n_q;
         if (!mbar_wait(q_empty + s, ((j / C::kStages) & 1) ^ 1, abort, a.status)) break;
 #ifdef ATTN_FAULT_INJECT
         if (blockIdx.x == 0 && blockIdx.y == 0 && j == a.fault_block) {  // the MMA warp's wait runs out
@@ -388,8 +373,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       return __all_sync(0xffffffffu, r);
     };
     for (int j = gg; j < n_it; j += 2) {
-      const int h = g * G + (j0 + j) / n_q;
-      const int q0 = (qt0 + (j0 + j) % n_q) * kBM;
+      const int h = g * G + j / n_q;
+      const int q0 = (qt0 + j % n_q) * kBM;
       const float* lse2 = a.lse2 + (static_cast<long long>(b) * a.Hq + h) * a.Sq_pad + q0;
       const float* dlt = a.delta + (static_cast<long long>(b) * a.Hq + h) * a.Sq_pad + q0;
       // Visible columns of this key's row form one window [cmin, cmax): query rows at or after the
@@ -487,30 +472,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     // dK / dV epilogue: TMEM rows -> bf16 global rows of this key tile (group 0: dV, group 1: dK);
     if (ok && n_it > 0) ok = wait_warp(all_done, 0);
     tc_fence_after();
-    // a split key tile's two parts add their fp32 rows into dkv_acc instead (dK scaled later)
-    const bool have = ok && n_it > 0;
-    const bool store = key < sp.Sk && (have || !split);
+    const bool store = key < sp.Sk;
+    const long long row = ((static_cast<long long>(sp.k0) + key) * a.Hkv + g) * D;
     const uint32_t col = gg == 0 ? C::kColDV : C::kColDK;
-    const float mul = (gg == 0 || split) ? 1.f : a.scale;
-    const long long row = split ? ((((static_cast<long long>(b) * a.Hkv + g) * a.n_split + kt) * 2 + gg) * kBN + t) * D
-                                : ((static_cast<long long>(sp.k0) + key) * a.Hkv + g) * D;
+    const float mul = gg == 0 ? 1.f : a.scale;
+    uint16_t* dst = (gg == 0 ? a.dv : a.dk) + row;
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 16) {
       uint32_t r[16];
-      if (have) {
+      if (ok && n_it > 0) {
         tmem_ld16(tmem + lane_addr + col + c0, r);
         tmem_wait_ld();
       } else {
 #pragma unroll
         for (int e = 0; e < 16; ++e) r[e] = 0u;
       }
-      if (!store) continue;
-      if (split) {
-        float* acc = a.dkv_acc + row + c0;
-#pragma unroll
-        for (int e = 0; e < 16; e += 4) red_add_v4_f32(acc + e, r + e);
-      } else {
-        uint16_t* dst = (gg == 0 ? a.dv : a.dk) + row + c0;
+      if (store) {
         uint4 w0, w1;
         w0.x = pack_bf16(__uint_as_float(r[0]) * mul, __uint_as_float(r[1]) * mul);
         w0.y = pack_bf16(__uint_as_float(r[2]) * mul, __uint_as_float(r[3]) * mul);
@@ -520,8 +497,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         w1.y = pack_bf16(__uint_as_float(r[10]) * mul, __uint_as_float(r[11]) * mul);
         w1.z = pack_bf16(__uint_as_float(r[12]) * mul, __uint_as_float(r[13]) * mul);
         w1.w = pack_bf16(__uint_as_float(r[14]) * mul, __uint_as_float(r[15]) * mul);
-        *reinterpret_cast<uint4*>(dst) = w0;
-        *reinterpret_cast<uint4*>(dst + 8) = w1;
+        *reinterpret_cast<uint4*>(dst + c0) = w0;
+        *reinterpret_cast<uint4*>(dst + c0 + 8) = w1;
       }
     }
   } else {
@@ -539,8 +516,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     for (int j = 0; j < n_it; ++j) {
       const int bb = j & 1;
-      const int h = g * G + (j0 + j) / n_q;
-      const int q0 = (qt0 + (j0 + j) % n_q) * kBM;
+      const int h = g * G + j / n_q;
+      const int q0 = (qt0 + j % n_q) * kBM;
       if (!wait_warp(dq_full + bb, (j >> 1) & 1)) break;
       tc_fence_after();
       // the whole dQ^T row of this lane (64 query columns) in one round trip; then its columns may
@@ -578,7 +555,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
                                                        const float* __restrict__ lse, float* __restrict__ lse2,
                                                        float* __restrict__ delta, float* __restrict__ dq_acc, int B,
                                                        int Hq, int Sq, int Sq_pad, const int* __restrict__ cu_q,
-                                                       int Tq, float* __restrict__ dkv_acc, long long dkv_n4) {
+                                                       int Tq) {
   constexpr int LPR = D / 8;     // lanes per row
   constexpr int RPW = 32 / LPR;  // rows per warp instruction
   constexpr int U = 4;           // row groups in flight per warp
@@ -641,14 +618,11 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
       }
     }
   }
-  // the whole accumulator (rows x D values, whatever its internal order) to zero, and the split key
-  // tiles' dK / dV accumulator
+  // the whole accumulator (rows x D values, whatever its internal order) to zero
   const long long n4 = rows * D / 4;
-  for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < n4 + dkv_n4;
-       t += static_cast<long long>(gridDim.x) * blockDim.x) {
-    float4* dst = t < n4 ? reinterpret_cast<float4*>(dq_acc) + t : reinterpret_cast<float4*>(dkv_acc) + (t - n4);
-    *dst = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
+  for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < n4;
+       t += static_cast<long long>(gridDim.x) * blockDim.x)
+    reinterpret_cast<float4*>(dq_acc)[t] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // dQ = scale * accumulator -> bf16. A thread takes four adjacent head-dim columns of one group of
@@ -692,47 +666,10 @@ __global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const float* __rest
   }
 }
 
-// dK, dV of the split key tiles: the fp32 sums of their two parts -> bf16 rows (dK times scale).
-// A thread takes four adjacent head-dim values of one key row.
-__global__ void __launch_bounds__(256) bwd_dkv_convert_kernel(const float* __restrict__ acc,
-                                                              uint16_t* __restrict__ dk, uint16_t* __restrict__ dv,
-                                                              int B, int Hkv, int Sk, int D, int n_split, float scale,
-                                                              const int* __restrict__ cu_k, int Tk) {
-  griddep_wait();  // the main kernel's partial sums are complete
-  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int qd = D / 4;
-  if (i >= static_cast<long long>(B) * Hkv * n_split * 2 * kBN * qd) return;
-  const int d4 = static_cast<int>(i % qd);
-  long long t = i / qd;
-  const int r = static_cast<int>(t % kBN);
-  t /= kBN;
-  const int which = static_cast<int>(t % 2);  // 0 dV, 1 dK
-  t /= 2;
-  const int kt = static_cast<int>(t % n_split);
-  t /= n_split;
-  const int g = static_cast<int>(t % Hkv);
-  const long long b = t / Hkv;
-  long long first = b * Sk;
-  int len = Sk;
-  if (cu_k) {
-    int f;
-    packed_rows(cu_k, static_cast<int>(b), Tk, Sk, f, len);
-    first = f;
-  }
-  const int key = kt * kBN + r;
-  if (key >= len) return;
-  const float4 x = reinterpret_cast<const float4*>(acc)[i];
-  const float mul = which ? scale : 1.f;
-  uint2 w;
-  w.x = pack_bf16(x.x * mul, x.y * mul);
-  w.y = pack_bf16(x.z * mul, x.w * mul);
-  *reinterpret_cast<uint2*>((which ? dk : dv) + ((first + key) * Hkv + g) * D + 4 * d4) = w;
-}
-
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 int pad128(int s) { return (s + 127) / 128 * 128; }
 
-template <int D>
+template <int D, bool PACKED>
 cudaError_t launch_bwd_sm100_d(const Problem& p, const void* q, const void* k, const void* v, const void* o,
                                const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
                                cudaStream_t st) {
@@ -742,30 +679,9 @@ cudaError_t launch_bwd_sm100_d(const Problem& p, const void* q, const void* k, c
   float* dq_acc = static_cast<float*>(workspace);
   float* lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(rows * D * 4));
   float* delta = reinterpret_cast<float*>(reinterpret_cast<char*>(lse2) + align256(rows * 4));
-  float* dkv_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(delta) + align256(rows * 4));
-  // Split the key tiles whose work (query tiles x heads of the group) exceeds 3/4 of the mean work
-  // per SM: under a causal mask the first key tiles see every query row, and one of them alone would
-  // outlast the other SMs' share. The causal work is counted at the longest sequence's lengths.
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int G = p.Hq / p.Hkv, n_kt = (p.Sk + kBN - 1) / kBN, n_qt = (p.Sq + kBM - 1) / kBM;
-  auto work = [&](int kt) {
-    int qt0 = 0;
-    if (p.causal) {
-      const int qmin = kt * kBN - (p.Sk - p.Sq);
-      qt0 = qmin <= 0 ? 0 : qmin / kBM;
-    }
-    return static_cast<long long>(G) * std::max(0, n_qt - qt0);
-  };
-  long long total = 0;
-  for (int kt = 0; kt < n_kt; ++kt) total += work(kt);
-  total *= static_cast<long long>(p.B) * p.Hkv;
-  const double mean = static_cast<double>(total) / std::max(1, sms);
-  int n_split = 0;
-  while (n_split < n_kt && work(n_split) >= 2 && work(n_split) > 0.75 * mean) ++n_split;
 
   CUtensorMap mq, mk, mv, mdo;
-  const bool packed = p.cu_q != nullptr;
+  constexpr bool packed = PACKED;
   const int mB = packed ? 1 : p.B, mSq = packed ? p.Tq : p.Sq, mSk = packed ? p.Tk : p.Sk;
   if (!make_map_bf16_sw128(&mq, q, mB, mSq, p.Hq, D, kBM) || !make_map_bf16_sw128(&mdo, dout, mB, mSq, p.Hq, D, kBM) ||
       !make_map_bf16_sw128(&mk, k, mB, mSk, p.Hkv, D, kBN) || !make_map_bf16_sw128(&mv, v, mB, mSk, p.Hkv, D, kBN))
@@ -777,12 +693,12 @@ cudaError_t launch_bwd_sm100_d(const Problem& p, const void* q, const void* k, c
     const unsigned blocks = static_cast<unsigned>(std::min<size_t>((rows + 63) / 64, 1u << 20));
     bwd_prep_kernel<D><<<blocks, 256, 0, st>>>(
         static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, lse2, delta, dq_acc, p.B, p.Hq,
-        p.Sq, Sq_pad, p.cu_q, p.Tq, dkv_acc, static_cast<long long>(p.B) * p.Hkv * n_split * 2 * kBN * D / 4);
+        p.Sq, Sq_pad, p.cu_q, p.Tq);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
-  e = cudaFuncSetAttribute(bwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  e = cudaFuncSetAttribute(bwd_sm100_kernel<D, PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   BwdArgs a;
   a.B = p.B;
@@ -809,12 +725,10 @@ cudaError_t launch_bwd_sm100_d(const Problem& p, const void* q, const void* k, c
 #else
   a.fault_block = -1;
 #endif
-  a.n_split = n_split;
-  a.dkv_acc = dkv_acc;
-  dim3 grid(p.Hkv * p.B, n_kt + n_split);
+  dim3 grid(p.Hkv * p.B, (p.Sk + kBN - 1) / kBN);
   {
     LaunchScope ls("bwd_sm100", st);
-    e = launch_dependent(bwd_sm100_kernel<D>, grid, dim3(kThreads), C::kSmemBytes, st, mq, mk, mv, mdo, a);
+    e = launch_dependent(bwd_sm100_kernel<D, PACKED>, grid, dim3(kThreads), C::kSmemBytes, st, mq, mk, mv, mdo, a);
   }
   if (e != cudaSuccess) return e;
   e = cudaGetLastError();
@@ -827,33 +741,27 @@ cudaError_t launch_bwd_sm100_d(const Problem& p, const void* q, const void* k, c
                          dq_acc, static_cast<uint16_t*>(dq), p.B, p.Hq, p.Sq, Sq_pad, D, p.scale, p.cu_q, p.Tq);
   }
   if (e != cudaSuccess) return e;
-  e = cudaGetLastError();
-  if (e != cudaSuccess || n_split == 0) return e;
-  const long long n_dkv = static_cast<long long>(p.B) * p.Hkv * n_split * 2 * kBN * (D / 4);
-  {
-    LaunchScope ls("bwd_dkv_convert", st);
-    e = launch_dependent(bwd_dkv_convert_kernel, dim3(static_cast<unsigned>((n_dkv + 255) / 256)), dim3(256), 0, st,
-                         dkv_acc, static_cast<uint16_t*>(dk), static_cast<uint16_t*>(dv), p.B, p.Hkv, p.Sk, D, n_split,
-                         p.scale, p.cu_k, p.Tk);
-  }
-  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 }  // namespace
 
 size_t bwd_sm100_workspace_bytes(int B, int Hq, int Hkv, int Sq, int Sk, int D) {
+  (void)Hkv;
+  (void)Sk;
   const size_t rows = static_cast<size_t>(B) * Hq * pad128(Sq);
-  // room for splitting every key tile (the host decides how many it splits per call)
-  const size_t dkv = static_cast<size_t>(B) * Hkv * ((Sk + kBN - 1) / kBN) * 2 * kBN * D * 4;
-  return align256(rows * D * 4) + 2 * align256(rows * 4) + align256(dkv);
+  return align256(rows * D * 4) + 2 * align256(rows * 4);
 }
 
 cudaError_t launch_bwd_sm100(const Problem& p, const void* q, const void* k, const void* v, const void* o,
                              const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
                              cudaStream_t st) {
-  if (p.D == 128) return launch_bwd_sm100_d<128>(p, q, k, v, o, lse, dout, dq, dk, dv, workspace, st);
-  return launch_bwd_sm100_d<64>(p, q, k, v, o, lse, dout, dq, dk, dv, workspace, st);
+  const bool packed = p.cu_q != nullptr;
+  if (p.D == 128)
+    return packed ? launch_bwd_sm100_d<128, true>(p, q, k, v, o, lse, dout, dq, dk, dv, workspace, st)
+                  : launch_bwd_sm100_d<128, false>(p, q, k, v, o, lse, dout, dq, dk, dv, workspace, st);
+  return packed ? launch_bwd_sm100_d<64, true>(p, q, k, v, o, lse, dout, dq, dk, dv, workspace, st)
+                : launch_bwd_sm100_d<64, false>(p, q, k, v, o, lse, dout, dq, dk, dv, workspace, st);
 }
 
 }  // namespace attn

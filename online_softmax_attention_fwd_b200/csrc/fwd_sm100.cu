@@ -13,7 +13,8 @@
 // same keys, and the CTA streams each 128-key K/V block once for both. When each key/value head
 // serves an even number of query heads, the two tiles are the same rows of two query heads of one
 // group: under a causal mask both then see the same number of blocks, and items come in 128-row
-// steps of length. Otherwise they are two consecutive row tiles of one head. Items are sorted
+// steps of length. Otherwise the item folds one head's row tiles: row tile n - 1 - r with row tile
+// r, so that under a causal mask a long tile shares its CTA with a short one. Items are sorted
 // longest first (under a causal mask the last rows see the most keys) and dealt to the CTAs in
 // snake order. Across
 // items the K/V ring runs on without a pause. The next item's Q is loaded as soon as the current
@@ -85,9 +86,9 @@ struct FwdArgs {
   float o_scale;     // O multiplier at the end (FP8: the V scale; 1 for bf16)
   // A work item is two 128-row query tiles that read the same K/V blocks. With head_pairs, the two
   // tiles are the same rows of query heads 2 hs and 2 hs + 1 (one key/value group, as the head
-  // count ratio is even); otherwise they are rows 256 s .. 256 s + 255 of one head.
+  // count ratio is even); otherwise they are row tiles n - 1 - r and r of one head (n row tiles).
   int head_pairs;
-  int n_slots;       // row positions per head set: 128-row tiles (head_pairs) or 256-row pairs
+  int n_slots;       // items per head set: row tiles (head_pairs) or folded pairs of row tiles
   int n_hsets;       // head sets per batch entry: Hq / 2 (head_pairs) or Hq
   uint16_t* o;
   float* lse;
@@ -108,16 +109,18 @@ struct FwdArgs {
 struct SeqSpan {
   int Sq, Sk, q0, k0;
 };
+template <bool PACKED>
 __device__ __forceinline__ SeqSpan seq_span(const FwdArgs& a, int b) {
-  if (a.cu_q) {
+  if constexpr (PACKED) {
     const int q0 = a.cu_q[b], q1 = a.cu_q[b + 1], k0 = a.cu_k[b], k1 = a.cu_k[b + 1];
     if (q0 < 0 || q1 < q0 || q1 > a.Tq || q1 - q0 > a.Sq || k0 < 0 || k1 < k0 || k1 > a.Tk || k1 - k0 > a.Sk) {
       record_status(a.status, kStatusBadArg);
       return SeqSpan{0, 0, 0, 0};
     }
     return SeqSpan{q1 - q0, k1 - k0, q0, k0};
+  } else {
+    return SeqSpan{a.Sq, a.Sk, b * a.Sq, b * a.Sk};
   }
-  return SeqSpan{a.Sq, a.Sk, b * a.Sq, b * a.Sk};
 }
 
 __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
@@ -147,7 +150,9 @@ __device__ __forceinline__ int fwd_item_index(int k, int c, int G, int n_items) 
 // One CTA per SM. Its 10 warps are dealt to the SM's four sub-partitions (three on some), and each
 // sub-partition has 16 K registers: at most 168 registers per thread, which the compiler derives
 // from these bounds.
-template <int D, bool F8>
+// Instantiated per element type (F8: e4m3), layout (PACKED: cu_seqlens offsets) and item shape (HP:
+// head pairs), so that each variant carries only its own index arithmetic.
+template <int D, bool F8, bool PACKED, bool HP>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
@@ -176,22 +181,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int BH = a.B * a.n_hsets;
   const int n_items = BH * a.n_slots;
   const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
-  // item i: row position n_slots - 1 - i / BH (the longest items first under a causal mask) of head
-  // set i % BH; tile t covers head h + t dh, rows q0 + t dq
-  const int dh = a.head_pairs ? 1 : 0, dq = a.head_pairs ? 0 : kBM;
+  // Item i of head set i % BH, rank r = i / BH (rank 0 the longest under a causal mask). Head
+  // pairs: both tiles are row tile n_slots - 1 - r of heads h and h + 1. Otherwise (one head): the
+  // item folds the sequence's row tiles, pairing tile n - 1 - r (rows q0, the longer) with tile r
+  // (rows q1), so that under a causal mask a long tile shares its CTA with a short one; the middle
+  // tile of an odd count runs alone, and ranks past the middle are empty.
+  constexpr int dh = HP ? 1 : 0;
   // TMA coordinates: dense tensors are 4-D maps (D, H, S, B); packed ones are (D, H, T, 1), where a
   // sequence's rows start at its first packed row (boxes may run into the next sequence's rows:
   // those keys are masked, their values weighted 0, and those query rows are not stored)
-  auto item_of = [&](int i, int& b, int& h, int& q0, int& n0, int& n1, SeqSpan& sp) {
-    const int bh = i % BH, slot = a.n_slots - 1 - i / BH;
+  auto item_of = [&](int i, int& b, int& h, int& q0, int& q1, int& n0, int& n1, SeqSpan& sp) {
+    const int bh = i % BH, r = i / BH;
     b = bh / a.n_hsets;
-    h = (bh % a.n_hsets) * (a.head_pairs ? 2 : 1);
-    q0 = slot * (a.head_pairs ? kBM : 2 * kBM);
-    sp = seq_span(a, b);
-    n0 = tile_blocks(sp, a.causal, q0);
-    n1 = tile_blocks(sp, a.causal, q0 + dq);
+    h = (bh % a.n_hsets) * (HP ? 2 : 1);
+    sp = seq_span<PACKED>(a, b);
+    if constexpr (HP) {
+      q0 = q1 = (a.n_slots - 1 - r) * kBM;
+      n0 = n1 = tile_blocks(sp, a.causal, q0);
+    } else {
+      const int nt = (sp.Sq + kBM - 1) / kBM, ta = nt - 1 - r;
+      q0 = ta * kBM;
+      q1 = r * kBM;
+      n0 = ta >= r ? tile_blocks(sp, a.causal, q0) : 0;
+      n1 = ta > r ? tile_blocks(sp, a.causal, q1) : 0;
+    }
   };
-  const bool packed = a.cu_q != nullptr;
+  constexpr bool packed = PACKED;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -239,9 +254,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int k = 0; ok; ++k) {
         const int i = fwd_item_index(k, cta, G, n_items);
         if (i < 0) break;
-        int b, h, q0, n0, n1;
+        int b, h, q0, q1, n0, n1;
         SeqSpan sp;
-        item_of(i, b, h, q0, n0, n1, sp);
+        item_of(i, b, h, q0, q1, n0, n1, sp);
         const int nmax = max(n0, n1);
         if (nmax == 0) continue;
         const int g = h / (a.Hq / a.Hkv);
@@ -255,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int at = 0; at < C::kAtoms; ++at)
             tma_load_4d(sQ + t * C::kTileBytes + at * kAtom, &tmQ, q_full, at * C::kAtomElts, h + t * dh,
-                        qrow0 + q0 + t * dq, bc);
+                        qrow0 + (t == 0 ? q0 : q1), bc);
         }
         ++qk;
         for (int j = 0; j < nmax; ++j) {
@@ -344,9 +359,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0; ok; ++k) {
       const int i = fwd_item_index(k, cta, G, n_items);
       if (i < 0) break;
-      int b, h, q0, n0, n1;
+      int b, h, q0, q1, n0, n1;
       SeqSpan sp;
-      item_of(i, b, h, q0, n0, n1, sp);
+      item_of(i, b, h, q0, q1, n0, n1, sp);
       const int nmax = max(n0, n1);
       if (nmax == 0) continue;
       const int nt[2] = {n0, n1};
@@ -437,12 +452,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0;; ++k) {
       const int i = fwd_item_index(k, cta, G, n_items);
       if (i < 0) break;
-      int b, h, q0, n0, n1;
+      int b, h, q0, q1, n0, n1;
       SeqSpan sp;
-      item_of(i, b, h, q0, n0, n1, sp);
+      item_of(i, b, h, q0, q1, n0, n1, sp);
       const int n_kv = t == 0 ? n0 : n1;
       h += t * dh;
-      const int qrow = q0 + t * dq + row;
+      const int qrow = (t == 0 ? q0 : q1) + row;
       int row_limit = sp.Sk - 1;  // largest visible key index for this row
       if (a.causal) row_limit = min(row_limit, qrow + sp.Sk - sp.Sq);
       float m = -INFINITY, l = 0.f;
@@ -541,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool have = ok && n_kv > 0;
       if (have) ok = wait_warp(o_done + t, ct & 1);
       tc_fence_after();
-      const float inv = l > 0.f ? a.o_scale / l : 0.f;
+      const float inv = l > 0.f ? (F8 ? a.o_scale : 1.f) / l : 0.f;
       const bool store = qrow < sp.Sq;
       uint16_t* orow = a.o + ((static_cast<long long>(sp.q0) + qrow) * a.Hq + h) * D;
       uint32_t orr[D];
@@ -592,12 +607,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------------------------
 // host side: tensor maps and launch
 // ---------------------------------------------------------------------------------------------
-template <int D, bool F8>
-cudaError_t launch_fwd_sm100_d(const Problem& p, const void* q, const void* k, const void* v, void* o, float* lse,
+template <int D, bool F8, bool PACKED, bool HP>
+cudaError_t launch_fwd_sm100_v(const Problem& p, const void* q, const void* k, const void* v, void* o, float* lse,
                                cudaStream_t st) {
   using C = FwdCfg<D, F8>;
   CUtensorMap mq, mk, mv;
-  const bool packed = p.cu_q != nullptr;
+  constexpr bool packed = PACKED;
   // packed batches: one sequence of Tq (Tk) rows as far as the maps are concerned
   const int mB = packed ? 1 : p.B, mSq = packed ? p.Tq : p.Sq, mSk = packed ? p.Tk : p.Sk;
   auto make = [&](CUtensorMap* m, const void* base, int S, int H, int rows) {
@@ -605,8 +620,8 @@ cudaError_t launch_fwd_sm100_d(const Problem& p, const void* q, const void* k, c
   };
   if (!make(&mq, q, mSq, p.Hq, kBM) || !make(&mk, k, mSk, p.Hkv, kBN) || !make(&mv, v, mSk, p.Hkv, kBN))
     return cudaErrorInvalidValue;
-  cudaError_t e =
-      cudaFuncSetAttribute(fwd_sm100_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(fwd_sm100_kernel<D, F8, PACKED, HP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::kSmemBytes);
   if (e != cudaSuccess) return e;
   FwdArgs a;
   a.B = p.B;
@@ -617,7 +632,7 @@ cudaError_t launch_fwd_sm100_d(const Problem& p, const void* q, const void* k, c
   a.causal = p.causal;
   a.scale_log2 = p.scale * p.qk_scale * kLog2e;
   a.o_scale = p.v_scale;
-  a.head_pairs = (p.Hq / p.Hkv) % 2 == 0 ? 1 : 0;
+  a.head_pairs = HP ? 1 : 0;
   a.n_slots = a.head_pairs ? (p.Sq + kBM - 1) / kBM : (p.Sq + 2 * kBM - 1) / (2 * kBM);
   a.n_hsets = a.head_pairs ? p.Hq / 2 : p.Hq;
   a.o = static_cast<uint16_t*>(o);
@@ -642,23 +657,35 @@ cudaError_t launch_fwd_sm100_d(const Problem& p, const void* q, const void* k, c
   dim3 grid(static_cast<unsigned>(std::min<long long>(n_items, sms)));
   {
     LaunchScope ls(F8 ? "fwd_sm100_fp8" : "fwd_sm100", st);
-    fwd_sm100_kernel<D, F8><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);
+    fwd_sm100_kernel<D, F8, PACKED, HP><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);
   }
   return cudaGetLastError();
 }
 
 }  // namespace
 
+// head pairs when each key/value head serves an even number of query heads
+template <int D, bool F8, bool PACKED>
+cudaError_t launch_fwd_sm100_d(const Problem& p, const void* q, const void* k, const void* v, void* o, float* lse,
+                               cudaStream_t st) {
+  if ((p.Hq / p.Hkv) % 2 == 0) return launch_fwd_sm100_v<D, F8, PACKED, true>(p, q, k, v, o, lse, st);
+  return launch_fwd_sm100_v<D, F8, PACKED, false>(p, q, k, v, o, lse, st);
+}
+
 cudaError_t launch_fwd_sm100(const Problem& p, const void* q, const void* k, const void* v, void* o, float* lse,
                              cudaStream_t st) {
-  if (p.D == 128) return launch_fwd_sm100_d<128, false>(p, q, k, v, o, lse, st);
-  return launch_fwd_sm100_d<64, false>(p, q, k, v, o, lse, st);
+  const bool packed = p.cu_q != nullptr;
+  if (p.D == 128)
+    return packed ? launch_fwd_sm100_d<128, false, true>(p, q, k, v, o, lse, st)
+                  : launch_fwd_sm100_d<128, false, false>(p, q, k, v, o, lse, st);
+  return packed ? launch_fwd_sm100_d<64, false, true>(p, q, k, v, o, lse, st)
+                : launch_fwd_sm100_d<64, false, false>(p, q, k, v, o, lse, st);
 }
 
 cudaError_t launch_fwd_sm100_fp8(const Problem& p, const void* q, const void* k, const void* v, void* o, float* lse,
                                  cudaStream_t st) {
-  if (p.D != 128) return cudaErrorInvalidValue;
-  return launch_fwd_sm100_d<128, true>(p, q, k, v, o, lse, st);
+  if (p.D != 128 || p.cu_q) return cudaErrorInvalidValue;
+  return launch_fwd_sm100_d<128, true, false>(p, q, k, v, o, lse, st);
 }
 
 }  // namespace attn

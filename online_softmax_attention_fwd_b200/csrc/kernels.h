@@ -141,8 +141,8 @@ cudaError_t launch_fwd_sm100_fp8(const Problem& p, const void* q, const void* k,
                                  cudaStream_t st);
 
 // bwd_sm100.cu: tcgen05 / TMA backward, bf16, D in {64, 128}; workspace = fp32 dQ accumulator
-// [B, Hq, Sq_pad, D] + lse2 [B, Hq, Sq_pad] + Delta [B, Hq, Sq_pad] + fp32 dK / dV of split key
-// tiles [B, Hkv, ceil(Sk / 128), 2, 128, D], each 256-byte aligned (Sq_pad = Sq rounded up to 128).
+// [B, Hq, Sq_pad, D] + lse2 [B, Hq, Sq_pad] + Delta [B, Hq, Sq_pad], each 256-byte aligned (Sq_pad =
+// Sq rounded up to 128).
 size_t bwd_sm100_workspace_bytes(int B, int Hq, int Hkv, int Sq, int Sk, int D);
 cudaError_t launch_bwd_sm100(const Problem& p, const void* q, const void* k, const void* v, const void* o,
                              const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,

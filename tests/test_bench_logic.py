@@ -39,3 +39,27 @@ def test_dominant_kernel_without_work_figure_claims_nothing(dom, bound):
 
 def test_no_profile_no_roofline():
     assert entry({}) is None
+
+
+def test_work_accounting():
+    # causal pairs: row i of an S x S causal problem sees i + 1 keys; Sq < Sk aligns bottom-right
+    assert bench.visible_pairs(4, 4, True) == 10 and bench.visible_pairs(4, 4, False) == 16
+    assert bench.visible_pairs(2, 5, True) == 4 + 5
+    assert bench.prefill_fwd_flops(1, 2, 4, 4, 8, True) == 4.0 * 8 * 2 * 10
+    # decode bytes: K and V once (bf16), Q read and O written (bf16), lse written (fp32)
+    assert bench.decode_bytes([3, 5], 4, 2, 8) == 2 * 8 * 2 * 8 * 2 + 2 * 4 * 8 * 2 * 2 + 2 * 4 * 4
+
+
+def test_reference_arm_counts_its_own_sample():
+    # the reference arm's value divides the sample's own FLOPs (one head of the prefill, fwd + 2.5x
+    # bwd, and the sampled streams' decode) by its measured seconds
+    class P:
+        q = type("T", (), {"shape": (1, 16, 4, 8)})()
+        k = type("T", (), {"shape": (1, 16, 2, 8)})()
+        causal = True
+
+    class Dc:
+        meta = {"lengths": [10, 20, 30]}
+
+    f = bench.oracle_sample_flops(P, Dc, 1, 2)
+    assert f == pytest.approx(3.5 * bench.prefill_fwd_flops(1, 1, 16, 16, 8, True) + 4.0 * 8 * 4 * 30)

@@ -141,8 +141,7 @@ attn_status_t attn_bwd_f32(const float* q, const float* k, const float* v, const
  *   their values weighted by 0, their query rows not stored), so those rows must hold finite values.
  *   D is 64 or 128. The backward's workspace: attn_bwd_varlen_workspace_size(B, Hq, Hkv,
  *   max_seqlen_q, max_seqlen_k, D) bytes, 256-byte aligned (fp32 dQ accumulator and per-row
- *   statistics, max_seqlen_q rows per sequence and head, and fp32 dK / dV room for the key tiles the
- *   kernel splits over two CTAs).
+ *   statistics, max_seqlen_q rows per sequence and head).
  * ------------------------------------------------------------------------------------------ */
 attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
                               const int* cu_seqlens_q, const int* cu_seqlens_k, int B,
@@ -244,7 +243,9 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* 
  *   q, o [N, q_len, Hq, D] bf16 (row (n, t, h) of o is the output of token t of stream n, head h);
  *   lse [N, Hq, q_len] fp32 (may be NULL); q_len >= 1, N * q_len * Hq < 2^31.
  *   k, v, kv_offsets, num_splits, max_splits, scale: as for attn_decode_splitkv (one split count per
- *   stream, shared by its tokens).
+ *   stream, shared by its tokens), except that with num_splits NULL and q_len > 1 the built-in rule
+ *   cuts about 512 keys per chunk: C(L) = min(max_splits, clamp(ceil(L/512), 2, 16)) (each chunk
+ *   carries q_len times the work; results differ from other split counts by rounding only).
  *   workspace: at least attn_decode_workspace_size(N * q_len, Hq, D, max_splits) bytes, 256-byte
  *   aligned.
  * attn_decode_paged_qlen: the same over a paged cache (arguments as attn_decode_paged).

@@ -548,8 +548,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Delta = rowsum(dO * O), lse2 = lse * log2(e) (+inf for rows that see no key), dQ accumulator = 0;
-// rows Sq .. Sq_pad - 1 are padding (lse2 = +inf, Delta = 0). A row (b, i, h) of the padded range is
-// D / 8 lanes, one 16-byte piece of O and dO each; a warp keeps four groups of rows in flight.
+// rows Sq .. Sq_pad - 1 of each sequence are padding (lse2 = +inf, Delta = 0). A warp takes eight
+// consecutive rows i .. i + 7 of one (b, h): D / 8 lanes per row, one 16-byte piece of O and of dO
+// each, all eight rows in flight; it then clears those rows' part of the interleaved accumulator,
+// two groups of four rows = 8 D contiguous floats.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                                                        const float* __restrict__ lse, float* __restrict__ lse2,
@@ -558,40 +560,33 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
                                                        int Tq) {
   constexpr int LPR = D / 8;     // lanes per row
   constexpr int RPW = 32 / LPR;  // rows per warp instruction
-  constexpr int U = 4;           // row groups in flight per warp
-  const long long rows = static_cast<long long>(B) * Sq_pad * Hq;  // (b, i, h), h fastest
+  constexpr int U = 8 / RPW;     // instructions for the warp's eight rows
   const int lane = threadIdx.x & 31, sub = lane / LPR, cl = lane % LPR;
   const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-  // row i of sequence b: its length and its row in the O / dO / lse layouts
-  auto span = [&](long long b, int& len, long long& first) {
+  const int chunks_per_bh = Sq_pad / 8;
+  const long long n_chunks = static_cast<long long>(B) * Hq * chunks_per_bh;
+  for (long long c = gw; c < n_chunks; c += nw) {
+    const long long bh = c / chunks_per_bh;
+    const int i0 = static_cast<int>(c % chunks_per_bh) * 8;
+    const int h = static_cast<int>(bh % Hq);
+    const long long b = bh / Hq;
+    long long first = b * Sq;  // the sequence's first row in O / dO
+    int len = Sq;
     if (cu_q) {
       int f;
       packed_rows(cu_q, static_cast<int>(b), Tq, Sq, f, len);
       first = f;
-    } else {
-      first = b * Sq;
-      len = Sq;
     }
-  };
-  for (long long r0 = gw * RPW * U; r0 < rows; r0 += nw * RPW * U) {
     uint4 x[U], y[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const long long row = r0 + u * RPW + sub;
-      const int h = static_cast<int>(row % Hq);
-      const int i = static_cast<int>((row / Hq) % Sq_pad);
-      const long long b = row / (static_cast<long long>(Hq) * Sq_pad);
+      const int i = i0 + u * RPW + sub;
       x[u] = y[u] = make_uint4(0u, 0u, 0u, 0u);
-      if (row < rows) {
-        int len;
-        long long first;
-        span(b, len, first);
-        if (i < len) {
-          const long long base = ((first + i) * Hq + h) * D + cl * 8;
-          x[u] = *reinterpret_cast<const uint4*>(o + base);
-          y[u] = *reinterpret_cast<const uint4*>(dout + base);
-        }
+      if (i < len) {
+        const long long base = ((first + i) * Hq + h) * D + cl * 8;
+        x[u] = *reinterpret_cast<const uint4*>(o + base);
+        y[u] = *reinterpret_cast<const uint4*>(dout + base);
       }
     }
 #pragma unroll
@@ -602,27 +597,21 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
       for (int e = 0; e < 4; ++e) sacc += bf16_lo(xs[e]) * bf16_lo(ys[e]) + bf16_hi(xs[e]) * bf16_hi(ys[e]);
 #pragma unroll
       for (int off = LPR / 2; off > 0; off >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, off);
-      const long long row = r0 + u * RPW + sub;
-      if (cl == 0 && row < rows) {
-        const int h = static_cast<int>(row % Hq);
-        const int i = static_cast<int>((row / Hq) % Sq_pad);
-        const long long b = row / (static_cast<long long>(Hq) * Sq_pad);
-        int len;
-        long long first;
-        span(b, len, first);
-        const long long li = (b * Hq + h) * Sq_pad + i;
+      if (cl == 0) {
+        const int i = i0 + u * RPW + sub;
+        const long long li = bh * Sq_pad + i;
         delta[li] = sacc;
         float l = -INFINITY;
-        if (i < len) l = cu_q ? lse[static_cast<long long>(h) * Tq + first + i] : lse[(b * Hq + h) * Sq + i];
+        if (i < len) l = cu_q ? lse[static_cast<long long>(h) * Tq + first + i] : lse[bh * Sq + i];
         lse2[li] = (l == -INFINITY) ? INFINITY : l * kLog2e;
       }
     }
+    // rows i0 .. i0 + 7 of (b, h) in the accumulator [B, Hq, Sq_pad / 4, D, 4]: 8 D floats from
+    // (bh Sq_pad / 4 + i0 / 4) D 4 on
+    float4* acc = reinterpret_cast<float4*>(dq_acc + (bh * (Sq_pad / 4) + i0 / 4) * D * 4);
+#pragma unroll
+    for (int e = lane; e < 2 * D; e += 32) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  // the whole accumulator (rows x D values, whatever its internal order) to zero
-  const long long n4 = rows * D / 4;
-  for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < n4;
-       t += static_cast<long long>(gridDim.x) * blockDim.x)
-    reinterpret_cast<float4*>(dq_acc)[t] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // dQ = scale * accumulator -> bf16. A thread takes four adjacent head-dim columns of one group of
@@ -689,7 +678,7 @@ cudaError_t launch_bwd_sm100_d(const Problem& p, const void* q, const void* k, c
 
   {
     LaunchScope ls("bwd_prep", st);
-    // rows / (8 warps x 2 or 4 rows x 4 groups) blocks, grid-strided
+    // one warp per eight rows (eight warps per block), grid-strided
     const unsigned blocks = static_cast<unsigned>(std::min<size_t>((rows + 63) / 64, 1u << 20));
     bwd_prep_kernel<D><<<blocks, 256, 0, st>>>(
         static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, lse2, delta, dq_acc, p.B, p.Hq,

@@ -39,9 +39,20 @@
 
 namespace attn {
 
-__host__ __device__ inline int decode_split_rule(int L, int max_splits) {
-  int c = (L + 255) / 256;
-  c = c < 4 ? 4 : (c > 16 ? 16 : c);
+// The built-in split count of a stream of L keys. One query token per stream: chunks of about 256
+// keys, 4 to 16 of them. Several tokens per stream: each chunk already carries q_len times the work
+// per key and its partial triples q_len times the bytes, so chunks of about 512 keys, 2 to 16 (the
+// 48-stream, four-token step took 140 us this way against 169 us with the one-token rule).
+__host__ __device__ inline int decode_split_rule(int L, int max_splits, int q_len = 1) {
+  int c, lo;
+  if (q_len <= 1) {
+    c = (L + 255) / 256;
+    lo = 4;
+  } else {
+    c = (L + 511) / 512;
+    lo = 2;
+  }
+  c = c < lo ? lo : (c > 16 ? 16 : c);
   if (c > max_splits) c = max_splits;
   return c < 1 ? 1 : c;
 }
@@ -57,12 +68,12 @@ size_t decode_workspace_bytes(int N, int Hq, int D, int max_splits) {
 
 namespace {
 
-__device__ __forceinline__ int stream_splits(const int* num_splits, int n, int L, int max_splits) {
+__device__ __forceinline__ int stream_splits(const int* num_splits, int n, int L, int max_splits, int q_len) {
   if (num_splits) {
     const int c = num_splits[n];
     return c < 1 ? 1 : (c > max_splits ? max_splits : c);
   }
-  return decode_split_rule(L, max_splits);
+  return decode_split_rule(L, max_splits, q_len);
 }
 
 // Where the keys of each stream live. Contiguous: stream n owns rows offsets[n] .. offsets[n+1] - 1
@@ -195,7 +206,7 @@ __device__ __forceinline__ bool dec_item(long long idx, int N, int Hq, int Hkv, 
   const int n = r / NG, gi = r - (r / NG) * NG;
   int start, L;
   dec_stream(kv, n, start, L);
-  const int C_n = stream_splits(num_splits, n, L, max_splits);
+  const int C_n = stream_splits(num_splits, n, L, max_splits, dq.q_len);
   if (c >= C_n) return false;
   dec_item_fill(n, c, gi, start, L, C_n, Hq, Hkv, dq, kv.block_table != nullptr, it);
   return true;
@@ -253,7 +264,7 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<RM>())
       if (n < N) {
         int st0, L;
         dec_stream(kv, n, st0, L);
-        cnt = NG * stream_splits(num_splits, n, L, max_splits);
+        cnt = NG * stream_splits(num_splits, n, L, max_splits, dq.q_len);
       }
       int incl = cnt;
 #pragma unroll
@@ -595,7 +606,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
   const int n = static_cast<int>(nt / q_len), tok = static_cast<int>(nt % q_len);
   int st0, L;
   dec_stream(kv, n, st0, L);
-  const int C = stream_splits(num_splits, n, L, max_splits);
+  const int C = stream_splits(num_splits, n, L, max_splits, q_len);
   const long long slot0 = gw * max_splits;
   // The first 16 partial rows are loaded before anything else, so their loads and those of the
   // (m, l) pairs are in flight together; lane c holds the pair of chunk c and c + 32 (max_splits

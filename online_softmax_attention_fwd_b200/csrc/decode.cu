@@ -26,9 +26,10 @@
 // copy ever touches memory past the caller's K and V buffers.
 // A paged cache (pages of a multiple of 16 keys, a block table per stream) runs through the same
 // kernels: chunks are then whole 16-key blocks, so a block lies in one page and its box starts at
-// the page's pool row; the stream's last partial block is copied row by row and the rest of it
-// zero-filled, since the rest of a page may hold anything. A page id outside the pool is not read:
-// its rows count as zeros and the device status records ATTN_ERR_INVALID_ARG.
+// the page's pool row. A stream's last block is copied whole too (the box stays inside its page),
+// and the consuming warp clears the V rows past the stream's end, since the rest of a page may hold
+// anything. A page id outside the pool is not read: its rows count as zeros and the device status
+// records ATTN_ERR_INVALID_ARG.
 #include <math.h>
 
 #include <algorithm>
@@ -85,6 +86,7 @@ struct DecKV {
   const int* seq_lens;
   const int* block_table;
   int max_pages, page_size, num_pages;
+  int page_shift;  // log2(page_size) when it is a power of two, else -1
 };
 
 __device__ __forceinline__ void dec_stream(const DecKV& kv, int n, int& start, int& L) {
@@ -226,7 +228,7 @@ __device__ __forceinline__ uint32_t dec_sw(int r, int d) {
   return (d >> 6) * kAtomBytes + sw128_offset(r, (d & 63) >> 3) + (d & 7) * 2;
 }
 
-template <int D, int RM>
+template <int D, int RM, bool PAGED>
 __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<RM>())
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
@@ -302,7 +304,7 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<RM>())
 
   if (warp == 4) {
     // ---------------------------------------------------------------- producer
-    const bool paged = kv.block_table != nullptr;
+    constexpr bool paged = PAGED;
     const int T = paged ? 0 : min(kv.offsets[N], kDecMapRows);  // no box may reach past the cache
     const long long rs = static_cast<long long>(Hkv) * D;
     const uint32_t qrow_bytes = static_cast<uint32_t>(dq.GT) * D * 2;  // one token's GT heads
@@ -332,14 +334,18 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<RM>())
         int row0, nrows;
         bool tile;
         if (paged) {
-          // chunks are whole blocks, so the block lies in one page; a full box is copied only when all
-          // of its rows are keys of the stream (the rest of a last page may hold anything)
-          const int page = kv.block_table[static_cast<long long>(it.n) * kv.max_pages + t0 / kv.page_size];
+          // chunks are whole blocks and pages a multiple of 16 keys, so the 16-row box lies inside
+          // one page and is always copied whole; the rows of a stream's last block past its end
+          // (which may hold anything, NaN included) are cleared in V by the consuming warp, and
+          // their scores are masked
+          const int pidx = kv.page_shift >= 0 ? t0 >> kv.page_shift : t0 / kv.page_size;
+          const int prow = kv.page_shift >= 0 ? t0 & (kv.page_size - 1) : t0 % kv.page_size;
+          const int page = kv.block_table[static_cast<long long>(it.n) * kv.max_pages + pidx];
           const bool page_ok = page >= 0 && page < kv.num_pages;
           if (!page_ok && lane == 0) record_status(status, kStatusBadArg);
-          row0 = page_ok ? page * kv.page_size + t0 % kv.page_size : 0;
-          tile = page_ok && t0 + kDecBlk <= it.k1;
-          nrows = page_ok ? min(kDecBlk, it.k1 - t0) : 0;  // an invalid page is read as zeros
+          row0 = page_ok ? page * kv.page_size + prow : 0;
+          tile = page_ok;
+          nrows = page_ok ? kDecBlk : 0;  // an invalid page is read as zeros
         } else {
           row0 = it.start + t0;
           tile = row0 + kDecBlk <= T;
@@ -443,6 +449,15 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<RM>())
       const uint32_t kb = smem_u32(sK + s * C::kBlkBytes);
       const uint32_t vb = smem_u32(sV + s * C::kBlkBytes);
       const int nk = min(kDecBlk, it.k1 - (it.k0 + bk * kDecBlk));  // keys of the chunk in this block
+      if (PAGED && nk < kDecBlk) {
+        // a paged block copied whole past its stream's end: V rows nk .. 15 to zero (the P V product
+        // reads them with probability 0, and 0 times NaN would not be 0)
+        for (int idx2 = lane; idx2 < (kDecBlk - nk) * (D / 8); idx2 += 32)
+          *reinterpret_cast<uint4*>(sV + s * C::kBlkBytes + dec_sw<D>(nk + idx2 / (D / 8), (idx2 % (D / 8)) * 8)) =
+              make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();  // before the stage's next copy, issued once this warp releases it
+        __syncwarp();
+      }
       // S^T for keys 0-7 (s0) and 8-15 (s1); rows g in s*[0..1], rows g + 8 in s*[2..3]
       float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -686,13 +701,13 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
     lse[(static_cast<long long>(n) * Hq + h) * q_len + tok] = Lt > 0.f ? (M + log2f(Lt)) * kLn2 : -INFINITY;
 }
 
-template <int D, int RM>
+template <int D, int RM, bool PAGED>
 cudaError_t launch_split(const DecodeProblem& p, const DecQ& dq, const void* q, const void* k, const void* v,
                          const CUtensorMap& mk, const CUtensorMap& mv, const DecKV& kv, const int* num_splits,
                          float* part_o, float* part_ml, cudaStream_t st) {
   using C = DecCfg<D, RM>;
   const int NG = p.Hkv * ((p.Hq / p.Hkv) / dq.GT) * dq.ntp;
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, RM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, RM, PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
   // a persistent grid: as many CTAs as fit on the SMs, capped by the number of item slots
@@ -706,7 +721,7 @@ cudaError_t launch_split(const DecodeProblem& p, const DecQ& dq, const void* q, 
       std::min<long long>(n_slots, static_cast<long long>(sms) * dec_ctas_per_sm<RM>()));
   {
     LaunchScope ls("decode_split", st);
-    decode_split_kernel<D, RM><<<grid, kDecThreads, C::kSmemBytes, st>>>(
+    decode_split_kernel<D, RM, PAGED><<<grid, kDecThreads, C::kSmemBytes, st>>>(
         mk, mv, static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v),
         kv, dq, p.N, num_splits, p.max_splits, p.Hq, p.Hkv, p.scale * kLog2e, part_o, part_ml,
         device_status_ptr());
@@ -753,8 +768,14 @@ cudaError_t launch_decode_d(const DecodeProblem& p, const void* q, const void* k
     return cudaErrorInvalidValue;
   int rm = 4;
   const DecQ dq = decode_rows(p.Hq / p.Hkv, p.q_len, rm);
-  cudaError_t e = rm == 4 ? launch_split<D, 4>(p, dq, q, k, v, mk, mv, kv, num_splits, part_o, part_ml, st)
-                          : launch_split<D, 16>(p, dq, q, k, v, mk, mv, kv, num_splits, part_o, part_ml, st);
+  // one instantiation per cache layout (packed / paged) and row variant
+  cudaError_t e;
+  if (kv.block_table)
+    e = rm == 4 ? launch_split<D, 4, true>(p, dq, q, k, v, mk, mv, kv, num_splits, part_o, part_ml, st)
+                : launch_split<D, 16, true>(p, dq, q, k, v, mk, mv, kv, num_splits, part_o, part_ml, st);
+  else
+    e = rm == 4 ? launch_split<D, 4, false>(p, dq, q, k, v, mk, mv, kv, num_splits, part_o, part_ml, st)
+                : launch_split<D, 16, false>(p, dq, q, k, v, mk, mv, kv, num_splits, part_o, part_ml, st);
   if (e != cudaSuccess) return e;
   const long long warps = static_cast<long long>(p.N) * p.q_len * p.Hq;
   {
@@ -773,7 +794,7 @@ cudaError_t launch_decode_d(const DecodeProblem& p, const void* q, const void* k
 cudaError_t launch_decode(const DecodeProblem& p, const void* q, const void* k, const void* v,
                           const int* kv_offsets, const int* num_splits, void* o, float* lse, void* workspace,
                           cudaStream_t st) {
-  const DecKV kv{kv_offsets, nullptr, nullptr, 0, 0, 0};
+  const DecKV kv{kv_offsets, nullptr, nullptr, 0, 0, 0, -1};
   if (p.D == 128) return launch_decode_d<128>(p, q, k, v, kv, kDecMapRows, num_splits, o, lse, workspace, st);
   return launch_decode_d<64>(p, q, k, v, kv, kDecMapRows, num_splits, o, lse, workspace, st);
 }
@@ -782,7 +803,10 @@ cudaError_t launch_decode_paged(const DecodeProblem& p, const void* q, const voi
                                 const int* block_table, int max_pages, const int* seq_lens, int page_size,
                                 int num_pages, const int* num_splits, void* o, float* lse, void* workspace,
                                 cudaStream_t st) {
-  const DecKV kv{nullptr, seq_lens, block_table, max_pages, page_size, num_pages};
+  int shift = -1;
+  for (int b = 4; b < 31; ++b)
+    if (page_size == (1 << b)) shift = b;
+  const DecKV kv{nullptr, seq_lens, block_table, max_pages, page_size, num_pages, shift};
   const long long rows = static_cast<long long>(num_pages) * page_size;
   if (p.D == 128) return launch_decode_d<128>(p, q, k_pages, v_pages, kv, rows, num_splits, o, lse, workspace, st);
   return launch_decode_d<64>(p, q, k_pages, v_pages, kv, rows, num_splits, o, lse, workspace, st);

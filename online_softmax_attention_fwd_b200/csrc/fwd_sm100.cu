@@ -471,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the whole 128-column row of S in registers: one round trip to TMEM
         uint32_t sr[kBN];
   #pragma unroll
-        for (int c = 0; c < kBN; c += 16) tmem_ld16(tS + c, sr + c);
+        for (int c = 0; c < kBN; c += 64) tmem_ld64(tS + c, sr + c);
         tmem_wait_ld();
         if (kbase + kBN - 1 > row_limit) {  // the block crosses this row's last visible key
   #pragma unroll
@@ -524,8 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (F8) {
             tmem_st16(tS + 16 * hf, pk);
           } else {
-            tmem_st16(tS + 32 * hf, pk);
-            tmem_st16(tS + 32 * hf + 16, pk + 16);
+            tmem_st32(tS + 32 * hf, pk);
           }
           // S of block j is complete, hence so is P V of block j - 1: O may be rescaled now, before
           // the first P V of block j is released.
@@ -562,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t orr[D];
       if (have && ok) {
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 16) tmem_ld16(tO + c0, orr + c0);
+        for (int c0 = 0; c0 < D; c0 += 64) tmem_ld64(tO + c0, orr + c0);
         tmem_wait_ld();
       } else {
 #pragma unroll

@@ -404,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         uint32_t sr[kBM];
 #pragma unroll
-        for (int c = 0; c < kBM; c += 16) tmem_ld16(tS + c, sr + c);
+        tmem_ld64(tS, sr);
         tmem_wait_ld();
 #pragma unroll
         for (int c4 = 0; c4 < kBM; c4 += 4) {
@@ -422,8 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[c / 2] = pack_bf16(p0, p1);
           }
         }
-        tmem_st16(tS, pk);
-        tmem_st16(tS + 16, pk + 16);
+        tmem_st32(tS, pk);
       }
       if (!wait_warp(dp_full + gg, (j >> 1) & 1)) {
         ok = false;
@@ -439,8 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         uint32_t dp[32];
-        tmem_ld16(tDP + hf * 32, dp);
-        tmem_ld16(tDP + hf * 32 + 16, dp + 16);
+        tmem_ld32(tDP + hf * 32, dp);
         tmem_wait_ld();
         uint32_t dk[16];
 #pragma unroll
@@ -524,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // be reused at once
       uint32_t r[kBM];
 #pragma unroll
-      for (int c = 0; c < kBM; c += 16) tmem_ld16(tmem + lane_addr + C::colDP(bb) + c, r + c);
+      tmem_ld64(tmem + lane_addr + C::colDP(bb), r);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();

@@ -24,10 +24,12 @@
 // the first 32 dP^T columns and into the tile's dS^T tile in shared memory, 128-byte swizzle). Then
 //   dV += P^T dO,  dK += dS^T Q              (A = P^T / dS^T in TMEM, B = dO / Q MN-major in SMEM)
 //   dQ^T = K^T dS^T                          (M = D, N = 64 query rows, K = 128 keys; both in SMEM)
-// Issue order for tile j: dV, then S^T of tile j + 2 over P^T (which dV has read), so the group
-// computes the next P^T while dK, dQ^T and the drain of this tile run; dK, then dQ^T over the dP^T
-// columns (which dK has read); dP^T of tile j + 2 once the drain has read dQ^T. MMAs execute in
-// issue order, which is what makes each overwrite in TMEM safe. dQ is produced transposed (head
+// Issue order for tile j: dV, dK, dQ^T over the dP^T columns (which dK has read), S^T of tile j + 2
+// over P^T (which dV has read; it keeps the tensor pipe busy while the drain reads dQ^T), and dP^T of
+// tile j + 2 once the drain has read dQ^T. MMAs execute in issue order, which is what makes each
+// overwrite in TMEM safe. The drain adds a tile's dQ into the accumulator only once that dP^T is
+// complete: its vector reductions use the same L1 data path as the tensor pipe's shared-memory
+// operand reads, and slowed the dP^T MMAs when the two ran at the same time. dQ is produced transposed (head
 // dim on the TMEM lanes, query rows on the columns), and the fp32 accumulator interleaves groups of
 // four query rows, [B, Hq, Sq_pad / 4, D, 4], so that a lane adds four consecutive rows of its
 // column with one 16-byte vector reduction and a warp instruction covers 512 contiguous bytes. For
@@ -322,13 +324,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < kBM / 16; ++kk)
           umma_ts_warp(tmem + C::kColDV, tmem + C::colS(bb) + kk * 8, sdesc_advance(dO, kk * 16 * 128), kIdG,
                        (j > 0 || kk > 0));
-        // S^T of tile j + 2 (same buffer) over P^T of tile j, which dV has just read: the group
-        // computes the next P^T while dK, dQ^T and the drain of this tile run
-        if (j + 2 < n_it) {
-          if (!wait(q_full + (j + 2) % C::kStages, ((j + 2) / C::kStages) & 1)) break;
-          tc_fence_after();
-          issue_scores(j + 2, kK, kQ, C::colS(bb), s_full + bb);
-        }
 #pragma unroll
         for (int kk = 0; kk < kBM / 16; ++kk)
           umma_ts_warp(tmem + C::kColDK, tmem + C::colDP(bb) + kk * 8, sdesc_advance(q, kk * 16 * 128), kIdG,
@@ -343,6 +338,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit_warp(ds_free + bb);
         umma_commit_warp(dq_full + bb);
         if (j + 2 < n_it) {
+          // S^T of tile j + 2 over P^T of tile j (dV has read it), while the drain reads dQ^T
+          if (!wait(q_full + (j + 2) % C::kStages, ((j + 2) / C::kStages) & 1)) break;
+          tc_fence_after();
+          issue_scores(j + 2, kK, kQ, C::colS(bb), s_full + bb);
           // dP^T of tile j + 2 over dQ^T of tile j, once the drain has read it
           if (!wait(dq_free + bb, (j >> 1) & 1)) break;
           tc_fence_after();
@@ -403,7 +402,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pk[kBM / 2];
       {
         uint32_t sr[kBM];
-#pragma unroll
         tmem_ld64(tS, sr);
         tmem_wait_ld();
 #pragma unroll
@@ -521,12 +519,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the whole dQ^T row of this lane (64 query columns) in one round trip; then its columns may
       // be reused at once
       uint32_t r[kBM];
-#pragma unroll
       tmem_ld64(tmem + lane_addr + C::colDP(bb), r);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_free + bb);
+      // the reductions wait until the dP^T MMAs that follow have finished reading shared memory
+      if (j + 2 < n_it && !wait_warp(dp_full + bb, ((j + 2) >> 1) & 1)) break;
       if (d < D) {  // at D = 64 warps 10 and 11 hold no dQ column
         // rows q0 + 4i .. q0 + 4i + 3 of column d: 16 contiguous bytes at acc + 4 D i
         float* acc = a.dq_acc + ((static_cast<long long>(b) * a.Hq + h) * a.Sq_pad + q0) * D + 4 * d;

@@ -10,7 +10,7 @@
  * unbounded or touches memory out of bounds, and the context stays usable.
  *
  *   family: 0 = attn_fwd's kernel (skips K block number `block` of CTA 0's ring),
- *           1 = attn_bwd's main kernel (skips Q/dO tile number `block` of CTA (0, 0)),
+ *           1 = attn_bwd's main kernel (skips Q/dO tile number `block` of CTA 0),
  *           2 = the split-KV decode's split kernel (skips ring block number `block` of CTA 0);
  *           -1 (or a negative block) switches injection off.
  * The setting is process-wide host state, read when each later call builds its kernel arguments.

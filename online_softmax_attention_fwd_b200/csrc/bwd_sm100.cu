@@ -10,9 +10,9 @@
 //   bwd_prep        Delta_i = dO_i . O_i, lse in base 2, and the fp32 dQ accumulator cleared, all
 //                   padded to a multiple of 128 query rows per (sequence, head) (padding rows:
 //                   lse2 = +inf, Delta = 0); packed batches get the longest sequence's padded rows;
-//   bwd_sm100       one CTA per (128-key tile, kv head): loops over the group's query heads x
-//                   64-row query tiles, keeps dK and dV for its keys in TMEM, and adds each tile's
-//                   dQ into the fp32 accumulator;
+//   bwd_sm100       one CTA per (128-key tile, kv head): loops over the group's 64-row query tiles
+//                   (from the last one down) x query heads, keeps dK and dV for its keys in TMEM,
+//                   and adds each tile's dQ into the fp32 accumulator;
 //   bwd_dq_convert  dQ = scale * accumulator, rounded to bf16.
 //
 // The main kernel works on transposed score tiles so that keys sit on the TMEM lanes:
@@ -103,7 +103,8 @@ struct BwdArgs {
   const int* cu_q;
   const int* cu_k;
   int Tq, Tk;
-  int fault_block;  // test-only fault-injection build: CTA (0, 0) skips this Q / dO tile (-1: none)
+  int fault_block;  // test-only fault-injection build: CTA 0 skips this Q / dO tile (-1: none)
+  int n_kt;         // key tiles per sequence (of the longest one in a packed batch)
 };
 
 // Rows first .. first + len - 1 of sequence b in a packed tensor of T rows: false (and an empty
@@ -158,7 +159,7 @@ __device__ __forceinline__ void red_add_v4_f32(float* p, const uint32_t* x) {
 
 // One CTA per SM. Its 14 warps put four on each of the SM's sub-partitions, and each sub-partition
 // has 16 K registers: at most 128 registers per thread, which the compiler derives from these bounds.
-template <int D, bool PACKED>
+template <int D, bool PACKED, bool SEQ_MAJOR>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -187,9 +188,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = static_cast<int>(blockIdx.x) % a.Hkv;
-  const int b = static_cast<int>(blockIdx.x) / a.Hkv;
-  const int kt = blockIdx.y;  // key tile; small indices carry the most work under a causal mask
+  // CTA -> (sequence b, kv head g, key tile kt); under a causal mask small kt carry the most work.
+  // Key tile by key tile over all sequences puts the heaviest CTAs first; sequence by sequence keeps
+  // the CTAs that run together on one sequence's Q / dO and dQ rows, for batches whose rows do not
+  // fit in L2 together (they would be streamed from DRAM once per wave of key tiles otherwise).
+  // Key tile by key tile: grid (B Hkv, key tiles). Sequence by sequence: a 1-D grid, kv head fastest.
+  const int bx = static_cast<int>(blockIdx.x);
+  const int g = bx % a.Hkv;
+  const int b = SEQ_MAJOR ? bx / (a.Hkv * a.n_kt) : bx / a.Hkv;
+  const int kt = SEQ_MAJOR ? (bx / a.Hkv) % a.n_kt : static_cast<int>(blockIdx.y);
   const int k0 = kt * kBN;
   const int G = a.Hq / a.Hkv;
   const BwdSpan sp = bwd_span<PACKED>(a, b);
@@ -205,7 +212,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     qt0 = qmin <= 0 ? 0 : qmin / kBM;
   }
   const int n_q = (k0 < sp.Sk && qt0 < n_qt_all) ? n_qt_all - qt0 : 0;
-  const int n_it = G * n_q;  // tiles: query head (slow) x query tile (fast)
+  // tiles: query tile (slow, from the last one down) x query head (fast). Every key tile's CTA then
+  // visits the query tiles in the same order, the last ones first, so the CTAs running at one time
+  // work on nearly the same Q / dO tiles and dQ accumulator rows, which stay in L2 between them.
+  const int n_it = G * n_q;
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -254,8 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued = 0;
       for (int j = 0; j < n_it; ++j) {
         const int s = j % C::kStages;
-        const int h = g * G + j / n_q;
-        const int qt = qt0 + j % n_q;
+        const int h = g * G + j % G;
+        const int qt = n_qt_all - 1 - j / G;
         if (!mbar_wait(q_empty + s, ((j / C::kStages) & 1) ^ 1, abort, a.status)) break;
 #ifdef ATTN_FAULT_INJECT
         if (blockIdx.x == 0 && blockIdx.y == 0 && j == a.fault_block) {  // the MMA warp's wait runs out
@@ -372,8 +382,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       return __all_sync(0xffffffffu, r);
     };
     for (int j = gg; j < n_it; j += 2) {
-      const int h = g * G + j / n_q;
-      const int q0 = (qt0 + j % n_q) * kBM;
+      const int h = g * G + j % G;
+      const int q0 = (n_qt_all - 1 - j / G) * kBM;
       const float* lse2 = a.lse2 + (static_cast<long long>(b) * a.Hq + h) * a.Sq_pad + q0;
       const float* dlt = a.delta + (static_cast<long long>(b) * a.Hq + h) * a.Sq_pad + q0;
       // Visible columns of this key's row form one window [cmin, cmax): query rows at or after the
@@ -512,8 +522,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     for (int j = 0; j < n_it; ++j) {
       const int bb = j & 1;
-      const int h = g * G + j / n_q;
-      const int q0 = (qt0 + j % n_q) * kBM;
+      const int h = g * G + j % G;
+      const int q0 = (n_qt_all - 1 - j / G) * kBM;
       if (!wait_warp(dq_full + bb, (j >> 1) & 1)) break;
       tc_fence_after();
       // the whole dQ^T row of this lane (64 query columns) in one round trip; then its columns may
@@ -684,7 +694,11 @@ cudaError_t launch_bwd_sm100_d(const Problem& p, const void* q, const void* k, c
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
-  e = cudaFuncSetAttribute(bwd_sm100_kernel<D, PACKED>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  e = cudaFuncSetAttribute(bwd_sm100_kernel<D, PACKED, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bwd_sm100_kernel<D, PACKED, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::kSmemBytes);
   if (e != cudaSuccess) return e;
   BwdArgs a;
   a.B = p.B;
@@ -711,10 +725,18 @@ cudaError_t launch_bwd_sm100_d(const Problem& p, const void* q, const void* k, c
 #else
   a.fault_block = -1;
 #endif
-  dim3 grid(p.Hkv * p.B, (p.Sk + kBN - 1) / kBN);
+  a.n_kt = (p.Sk + kBN - 1) / kBN;
+  // Q, dO (bf16) and the dQ accumulator (fp32) of the whole batch: sequence by sequence once they
+  // would take more than half of the 126 MB L2
+  const double rows_bytes = static_cast<double>(p.B) * p.Hq * D * (4.0 * p.Sq + 4.0 * Sq_pad);
+  const bool seq_major = p.B > 1 && rows_bytes > 64.0 * 1024 * 1024;
   {
     LaunchScope ls("bwd_sm100", st);
-    e = launch_dependent(bwd_sm100_kernel<D, PACKED>, grid, dim3(kThreads), C::kSmemBytes, st, mq, mk, mv, mdo, a);
+    e = seq_major ? launch_dependent(bwd_sm100_kernel<D, PACKED, true>,
+                                     dim3(static_cast<unsigned>(static_cast<long long>(p.Hkv) * p.B * a.n_kt)),
+                                     dim3(kThreads), C::kSmemBytes, st, mq, mk, mv, mdo, a)
+                  : launch_dependent(bwd_sm100_kernel<D, PACKED, false>, dim3(p.Hkv * p.B, a.n_kt), dim3(kThreads),
+                                     C::kSmemBytes, st, mq, mk, mv, mdo, a);
   }
   if (e != cudaSuccess) return e;
   e = cudaGetLastError();

@@ -80,7 +80,7 @@ def test_backward_wait_runs_out_then_recovers(through):
     dev = torch.device("cuda")
     q, k, v, do = (t.to(dev) for t in (w.q, w.k, w.v, w.do))
     o, lse = attn.fwd(q, k, v, causal=True, scale=w.scale)
-    L.attn_fault_inject(1, 5)            # CTA (0, 0) never loads its sixth Q / dO tile
+    L.attn_fault_inject(1, 5)            # CTA 0 never loads its sixth Q / dO tile
     attn.bwd(q, k, v, o, lse, do, causal=True, scale=w.scale)
     torch.cuda.synchronize()
     assert _status(L) == TIMEOUT

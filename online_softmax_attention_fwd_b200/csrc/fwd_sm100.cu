@@ -56,6 +56,12 @@ constexpr int kBM = 128;   // query rows per tile (two tiles per CTA)
 constexpr int kBN = 128;   // keys per block
 constexpr int kThreads = 320;
 constexpr int kAtom = 128 * 128;  // 128 rows x 128 bytes (16 KB)
+// Packed batches: shared-memory tables for the item list (sequence lengths, sequences by length,
+// item counts per rank), for up to kMaxSeqs sequences and kMaxSlots ranks; beyond that every
+// (sequence, rank) pair stays an item and the empty ones are skipped.
+constexpr int kMaxSeqs = 1024;
+constexpr int kMaxSlots = 2048;
+constexpr int kTabBytes = (2 * kMaxSeqs + kMaxSlots + 1) * 4;
 
 // F8: e4m3 Q, K, V (one byte per element, D = 128 only) instead of bf16.
 template <int D, bool F8 = false>
@@ -100,6 +106,7 @@ struct FwdArgs {
   const int* cu_k;
   int Tq, Tk;
   int fault_block;  // test-only fault-injection build: CTA 0 skips this K load (-1: none)
+  int compact;      // packed batches: deal only the items that exist (tables in shared memory)
 };
 
 // Lengths and first packed rows of sequence b (dense: every sequence has Sq / Sk rows). Offsets
@@ -179,8 +186,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = a.B * a.n_hsets;
-  const int n_items = BH * a.n_slots;
   const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
+  // packed item tables (after the barriers and the rest of the per-CTA state)
+  int* s_len = reinterpret_cast<int*>(smem + C::kOffMisc + 64);  // [kMaxSeqs] query rows of each sequence
+  int* s_order = s_len + kMaxSeqs;                                // [kMaxSeqs] sequences, longest first
+  int* s_pref = s_order + kMaxSeqs;                               // [n_slots + 1] items before rank r
+  const bool compact = PACKED && a.compact;
   // Item i of head set i % BH, rank r = i / BH (rank 0 the longest under a causal mask). Head
   // pairs: both tiles are row tile n_slots - 1 - r of heads h and h + 1. Otherwise (one head): the
   // item folds the sequence's row tiles, pairing tile n - 1 - r (rows q0, the longer) with tile r
@@ -190,10 +201,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   // TMA coordinates: dense tensors are 4-D maps (D, H, S, B); packed ones are (D, H, T, 1), where a
   // sequence's rows start at its first packed row (boxes may run into the next sequence's rows:
   // those keys are masked, their values weighted 0, and those query rows are not stored)
+  // With the packed tables, the items are only the (sequence, rank) pairs with rows: rank by rank,
+  // and within a rank the sequences longest first, head sets fastest.
   auto item_of = [&](int i, int& b, int& h, int& q0, int& q1, int& n0, int& n1, SeqSpan& sp) {
-    const int bh = i % BH, r = i / BH;
-    b = bh / a.n_hsets;
-    h = (bh % a.n_hsets) * (HP ? 2 : 1);
+    int r, hs;
+    if (compact) {
+      int lo = 0, hi = a.n_slots - 1;  // the last rank whose first item is at or before i
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_pref[mid] <= i) lo = mid;
+        else hi = mid - 1;
+      }
+      r = lo;
+      const int w = i - s_pref[r];
+      b = s_order[w / a.n_hsets];
+      hs = w % a.n_hsets;
+    } else {
+      const int bh = i % BH;
+      r = i / BH;
+      b = bh / a.n_hsets;
+      hs = bh % a.n_hsets;
+    }
+    h = hs * (HP ? 2 : 1);
     sp = seq_span<PACKED>(a, b);
     if constexpr (HP) {
       q0 = q1 = (a.n_slots - 1 - r) * kBM;
@@ -239,10 +268,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
+  if (compact) {
+    // lengths (a sequence with offsets outside the tensors counts as empty), then each sequence's
+    // place in the order longest first, and the items of each rank: the sequences long enough to
+    // have that rank (a prefix of the order), times the head sets
+    for (int b = threadIdx.x; b < a.B; b += kThreads) s_len[b] = seq_span<PACKED>(a, b).Sq;
+    __syncthreads();
+    for (int b = threadIdx.x; b < a.B; b += kThreads) {
+      const int L = s_len[b];
+      int rank = 0;
+      for (int o = 0; o < a.B; ++o) rank += (s_len[o] > L) || (s_len[o] == L && o < b);
+      s_order[rank] = b;
+    }
+    for (int r = threadIdx.x; r < a.n_slots; r += kThreads) {
+      int cnt = 0;
+      for (int o = 0; o < a.B; ++o) {
+        const int nt = (s_len[o] + kBM - 1) / kBM;  // the sequence's row tiles
+        cnt += HP ? (a.n_slots - 1 - r) < nt : 2 * r + 1 <= nt;
+      }
+      s_pref[r + 1] = cnt * a.n_hsets;
+    }
+    __syncthreads();
+    if (warp == 0) {  // running sum over the ranks, 32 at a time
+      int carry = 0;
+      if (lane == 0) s_pref[0] = 0;
+      for (int base = 1; base <= a.n_slots; base += 32) {
+        const int idx = base + lane;
+        int v = idx <= a.n_slots ? s_pref[idx] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= o) v += u;
+        }
+        v += carry;
+        if (idx <= a.n_slots) s_pref[idx] = v;
+        carry = __shfl_sync(0xffffffffu, v, 31);
+      }
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  const int n_items = compact ? s_pref[a.n_slots] : BH * a.n_slots;
 
   if (warp == 8) {
     // ------------------------------------------------------------------ TMA producer
@@ -610,6 +678,8 @@ template <int D, bool F8, bool PACKED, bool HP>
 cudaError_t launch_fwd_sm100_v(const Problem& p, const void* q, const void* k, const void* v, void* o, float* lse,
                                cudaStream_t st) {
   using C = FwdCfg<D, F8>;
+  constexpr int kSmem = C::kSmemBytes + (PACKED ? kTabBytes : 0);
+  static_assert(kSmem <= 232448, "shared memory per CTA");
   CUtensorMap mq, mk, mv;
   constexpr bool packed = PACKED;
   // packed batches: one sequence of Tq (Tk) rows as far as the maps are concerned
@@ -620,7 +690,7 @@ cudaError_t launch_fwd_sm100_v(const Problem& p, const void* q, const void* k, c
   if (!make(&mq, q, mSq, p.Hq, kBM) || !make(&mk, k, mSk, p.Hkv, kBN) || !make(&mv, v, mSk, p.Hkv, kBN))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(fwd_sm100_kernel<D, F8, PACKED, HP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::kSmemBytes);
+                                       kSmem);
   if (e != cudaSuccess) return e;
   FwdArgs a;
   a.B = p.B;
@@ -646,6 +716,7 @@ cudaError_t launch_fwd_sm100_v(const Problem& p, const void* q, const void* k, c
 #else
   a.fault_block = -1;
 #endif
+  a.compact = packed && p.B <= kMaxSeqs && a.n_slots <= kMaxSlots;
   // a persistent grid: one CTA per SM, each walking its share of the (head, tile pair) items
   int dev = 0, sms = 0;
   e = cudaGetDevice(&dev);
@@ -656,7 +727,7 @@ cudaError_t launch_fwd_sm100_v(const Problem& p, const void* q, const void* k, c
   dim3 grid(static_cast<unsigned>(std::min<long long>(n_items, sms)));
   {
     LaunchScope ls(F8 ? "fwd_sm100_fp8" : "fwd_sm100", st);
-    fwd_sm100_kernel<D, F8, PACKED, HP><<<grid, kThreads, C::kSmemBytes, st>>>(mq, mk, mv, a);
+    fwd_sm100_kernel<D, F8, PACKED, HP><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, a);
   }
   return cudaGetLastError();
 }

@@ -52,6 +52,24 @@ def test_varlen_matches_oracle(lq, lk, Hq, Hkv, D, causal):
     check(W.packed_prefill(lq, lk, Hq, Hkv, D, causal, seed=sum(lq) + sum(lk) + D))
 
 
+@pytest.mark.parametrize("lq,Hq,Hkv,D", [
+    ([700, 5, 300, 0, 256, 255, 129, 1, 640], 3, 1, 64),     # single-head items, ranks of many sizes
+    ([1000, 3, 0, 517, 129, 128, 127, 1], 8, 2, 128),        # head pairs
+])
+def test_varlen_item_list_skips_missing_ranks(lq, Hq, Hkv, D):
+    # the forward deals only the (sequence, rank) items that exist, longest first: every sequence's
+    # rows still come out, whatever the spread of lengths
+    check(W.packed_prefill(lq, lq, Hq, Hkv, D, True, seed=sum(lq) + Hq))
+
+
+def test_varlen_more_sequences_than_the_item_tables():
+    # 1100 short sequences (more than the forward's shared-memory item tables hold): every
+    # (sequence, rank) pair stays an item and the empty ones are skipped
+    rng = np.random.default_rng(11)
+    lq = [int(x) for x in rng.integers(0, 7, 1100)]
+    check(W.packed_prefill(lq, lq, 2, 1, 64, True, seed=11))
+
+
 def test_varlen_equal_lengths_equal_dense_call():
     # the same batch packed and dense gives bit-identical forward results and gradients
     wd = W.random_prefill(3, 384, 384, 8, 2, 128, True, seed=5)

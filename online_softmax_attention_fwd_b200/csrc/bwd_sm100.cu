@@ -584,6 +584,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
       int f;
       packed_rows(cu_q, static_cast<int>(b), Tq, Sq, f, len);
       first = f;
+      // the main kernel reads rows of the sequence's 64-row query tiles only
+      if (i0 >= (len + 63) / 64 * 64) continue;
     }
     uint4 x[U], y[U];
 #pragma unroll

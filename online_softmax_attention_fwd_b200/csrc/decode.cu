@@ -129,8 +129,11 @@ struct DecCfg {
   static constexpr int kBlkBytes = kAtoms * kAtomBytes;  // 16 key rows x D bf16
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kDecStages * kBlkBytes;
-  static constexpr int kOffQ = 2 * kDecStages * kBlkBytes;  // [2 items][RM rows][D] bf16
-  static constexpr int kQBuf = RM * D * 2;
+  static constexpr int kOffQ = 2 * kDecStages * kBlkBytes;  // [2 items][RM rows][D + 8] bf16
+  // Query rows 16 bytes apart beyond their D elements: the compute warps' fragment loads (eight
+  // rows, four consecutive words each) then fall on 32 different banks instead of four.
+  static constexpr int kQRow = D * 2 + 16;
+  static constexpr int kQBuf = RM * kQRow;
   static constexpr int kOffDep = kOffQ + 2 * kQBuf;         // warps 1-3: [3][RM rows][D] fp32
   static constexpr int kOffBar = kOffDep + 3 * RM * D * 4;
   static constexpr int kNumBars = 2 * kDecStages + 4;       // full, empty, q_full[2], q_empty[2]
@@ -320,9 +323,10 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<RM>())
           const int ntok = min(dq.TQ, dq.q_len - it.tq0);
           mbar_arrive_expect_tx(q_full + (qi & 1), ntok * qrow_bytes);
           for (int t = 0; t < ntok; ++t)
-            bulk_load(sQ + (qi & 1) * C::kQBuf + t * qrow_bytes,
-                      q + ((static_cast<long long>(it.n) * dq.q_len + it.tq0 + t) * Hq + it.h0) * D, qrow_bytes,
-                      q_full + (qi & 1));
+            for (int hh = 0; hh < dq.GT; ++hh)
+              bulk_load(sQ + (qi & 1) * C::kQBuf + (t * dq.GT + hh) * C::kQRow,
+                        q + ((static_cast<long long>(it.n) * dq.q_len + it.tq0 + t) * Hq + it.h0 + hh) * D, D * 2,
+                        q_full + (qi & 1));
         }
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -429,7 +433,7 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<RM>())
       const int row = gq + 8 * r;
       valid[r] = row < nrow && row < RM;
       lim[r] = it.L - dq.q_len + it.tq0 + row / dq.GT - it.k0;
-      qrow[r] = reinterpret_cast<const uint32_t*>(sQ + qbuf * C::kQBuf) + (valid[r] ? row : 0) * (D / 2);
+      qrow[r] = reinterpret_cast<const uint32_t*>(sQ + qbuf * C::kQBuf + (valid[r] ? row : 0) * C::kQRow);
     }
     float o[D / 8][4];
 #pragma unroll

@@ -565,6 +565,10 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
                                                        float* __restrict__ delta, float* __restrict__ dq_acc, int B,
                                                        int Hq, int Sq, int Sq_pad, const int* __restrict__ cu_q,
                                                        int Tq) {
+  // The main kernel may be placed as soon as every block of this grid has started (it waits for
+  // this grid's results with griddepcontrol.wait): its set-up and first score MMAs then overlap
+  // this kernel's last blocks.
+  griddep_launch_dependents();
   constexpr int LPR = D / 8;     // lanes per row
   constexpr int RPW = 32 / LPR;  // rows per warp instruction
   constexpr int U = 8 / RPW;     // instructions for the warp's eight rows

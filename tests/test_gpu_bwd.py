@@ -71,6 +71,15 @@ def test_odd_shapes(B, Sq, Sk, Hq, Hkv, D, causal):
 
 
 @pytest.mark.parametrize("B,Sq,Sk,Hq,Hkv,D,causal", [
+    (3, 2048, 2048, 16, 4, 128, True), (5, 2048, 2048, 16, 16, 64, False)])
+def test_large_batches_run_sequence_by_sequence(B, Sq, Sk, Hq, Hkv, D, causal):
+    # batches whose Q, dO and dQ accumulator rows exceed half of L2 take the sequence-by-sequence
+    # CTA order (a second instantiation of the backward kernel)
+    assert B * Hq * D * (4 * Sq + 4 * ((Sq + 127) // 128 * 128)) > 64 * 1024 * 1024
+    check_bwd(W.random_prefill(B, Sq, Sk, Hq, Hkv, D, causal, seed=B + Sq + D))
+
+
+@pytest.mark.parametrize("B,Sq,Sk,Hq,Hkv,D,causal", [
     (1, 77, 77, 3, 1, 40, True), (2, 50, 90, 2, 2, 256, False), (1, 33, 20, 4, 2, 64, True)])
 def test_fp32_any_head_dim(B, Sq, Sk, Hq, Hkv, D, causal):
     w = W.random_prefill(B, Sq, Sk, Hq, Hkv, D, causal, dtype=torch.float32, seed=9)

@@ -97,11 +97,19 @@ def _check(fn: str, status: int) -> None:
 
 
 def _ptr(t: Optional[torch.Tensor]):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    # a plain int: ctypes passes it as the declared void* without building a c_void_p object
+    return None if t is None else t.data_ptr()
+
+
+# torch's raw current-stream query skips building a Stream object (about 3 us per call); the public
+# call is the fallback where it is missing
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
 
 
 def _stream():
-    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if _raw_stream is not None:
+        return _raw_stream(torch.cuda.current_device())
+    return torch.cuda.current_stream().cuda_stream
 
 
 def _expect(t: torch.Tensor, name: str, dtype, ndim: int):

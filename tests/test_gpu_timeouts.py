@@ -111,3 +111,45 @@ def test_decode_wait_runs_out_then_recovers(through):
     o_ref, lse_ref = oracle.decode_attention(np64(w.q), np64(w.k), np64(w.v), w.offsets.numpy(), w.scale)
     assert_o_bf16(np64(o), o_ref)
     assert_lse(np64(lse), lse_ref)
+
+
+def test_packed_forward_wait_runs_out_then_recovers(through):
+    # the packed forward (item list built in shared memory) takes the same unwind path
+    L = through
+    w = W.packed_prefill([300, 0, 700, 129], [300, 0, 700, 129], 4, 2, 128, True, seed=54)
+    dev = torch.device("cuda")
+    q, k, v, cq, ck = (t.to(dev) for t in (w.q, w.k, w.v, w.cu_q, w.cu_k))
+    L.attn_fault_inject(0, 2)
+    attn.fwd_varlen(q, k, v, cq, ck, 700, 700, causal=True, scale=w.scale)
+    torch.cuda.synchronize()
+    assert _status(L) == TIMEOUT
+    assert _status(L) == 0
+    L.attn_fault_inject(-1, -1)
+    o, lse = attn.fwd_varlen(q, k, v, cq, ck, 700, 700, causal=True, scale=w.scale)
+    torch.cuda.synchronize()
+    assert _status(L) == 0
+    o_ref, lse_ref = oracle.attention_fwd_varlen(np64(w.q), np64(w.k), np64(w.v), w.cu_q.numpy(), w.cu_k.numpy(),
+                                                 True, w.scale)
+    assert_o_bf16(np64(o), o_ref)
+    assert_lse(np64(lse), lse_ref)
+
+
+def test_sequence_order_backward_wait_runs_out_then_recovers(through):
+    # a batch large enough for the backward's sequence-by-sequence CTA order
+    L = through
+    w = W.random_prefill(3, 2048, 2048, 16, 4, 128, True, seed=55)
+    dev = torch.device("cuda")
+    q, k, v, do = (t.to(dev) for t in (w.q, w.k, w.v, w.do))
+    o, lse = attn.fwd(q, k, v, causal=True, scale=w.scale)
+    L.attn_fault_inject(1, 5)
+    attn.bwd(q, k, v, o, lse, do, causal=True, scale=w.scale)
+    torch.cuda.synchronize()
+    assert _status(L) == TIMEOUT
+    assert _status(L) == 0
+    L.attn_fault_inject(-1, -1)
+    dq, dk, dv = attn.bwd(q, k, v, o, lse, do, causal=True, scale=w.scale)
+    torch.cuda.synchronize()
+    assert _status(L) == 0
+    refs = oracle.attention_bwd(np64(w.q), np64(w.k), np64(w.v), np64(w.do), True, w.scale)
+    for name, g, r in zip(("dQ", "dK", "dV"), (dq, dk, dv), refs):
+        assert_grad_bf16(np64(g), r, name)
